@@ -1,0 +1,159 @@
+/*
+ * bitlinear.h -- C ABI of the B200 (sm_100a) Sparse-BitNet BitLinear path.
+ *
+ * One BitLinear layer: a dynamic N:M mask over the latent fp32 weights, absmean
+ * ternary codes {-1, 0, +1}, per-token int8 activations, the masked ternary x int8
+ * product with int32 accumulation, and the dual straight-through backward.
+ *
+ * Sources (pages named by title and section):
+ *   - Sparse-BitNet article (m.top168.com/news/show-814037), section 三: the mask is
+ *     recomputed every training step; the dual straight-through estimator passes
+ *     gradients through quantiser and mask; masked weights still get gradients.
+ *     Section 五: one threshold per group of 8 weights. Section 六: quantise first,
+ *     then sparsify; the mask ranks the full-precision latent weights.
+ *   - Sparse-BitNet paper digest (shd-paper.top), abstract: 1.58-bit weights with
+ *     dynamic N:M sparsity, run on a custom sparse tensor-core operator.
+ *   - BitNet b1.58 2B4T article (lsdiaocha.cn/2025/0716/3169029), section 一:
+ *     absmean quantisation of the weights to {-1, 0, +1}, 8-bit integer activations,
+ *     BitLinear layers without bias. Section 四: four ternary values per byte, moved
+ *     HBM -> shared memory and unpacked before the product with int8 activations.
+ *
+ * Conventions shared by every entry point:
+ *   - Memory: every pointer is a DEVICE pointer owned by the caller; the library
+ *     allocates no device memory. All arrays are row-major and contiguous. Every
+ *     pointer must be 16-byte aligned (BL_ERR_ALIGNMENT otherwise).
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Calls only enqueue work and return; results are ready when the
+ *     stream reaches them.
+ *   - Shapes: k_in % 64 == 0, 64 <= k_in <= 131072, n_out % 16 == 0, n_out >= 16,
+ *     t >= 0 (t = 0 is a valid empty batch). Else BL_ERR_UNSUPPORTED_SHAPE.
+ *   - bf16 arrays are passed as uint16_t bit patterns.
+ *   - Errors: argument, shape and alignment errors return before anything is
+ *     enqueued; a failed launch returns BL_ERR_CUDA. bitlinear_last_error() gives a
+ *     message for the last non-OK status of the calling thread.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BL_OK = 0,
+  BL_ERR_INVALID_ARG = -1,       /* null pointer, bad N:M, bad dtype            */
+  BL_ERR_UNSUPPORTED_SHAPE = -2, /* shape outside the rules above               */
+  BL_ERR_ALIGNMENT = -3,         /* a pointer is not 16-byte aligned            */
+  BL_ERR_RANGE = -4,             /* a latent weight is non-finite or |w| >= 2^16 */
+  BL_ERR_CUDA = -5,              /* a CUDA call or kernel launch failed          */
+  BL_ERR_TIMEOUT = -6,           /* a kernel gave up on a bounded wait          */
+  BL_ERR_WORKSPACE = -7          /* workspace missing or too small               */
+} bl_status;
+
+typedef enum { BL_OUT_BF16 = 0, BL_OUT_F32 = 1 } bl_dtype;
+
+/* Bytes of workspace bitlinear_quant_mask needs for a [n_out, k_in] tensor. */
+size_t bitlinear_quant_mask_workspace_size(int64_t n_out, int64_t k_in);
+
+/*
+ * Steps a1 + a2: absmean scale, N:M mask and masked ternary codes of one latent
+ * weight tensor W [n_out, k_in] (fp32). Recompute it every training step.
+ *
+ *   gamma   = mean|W| + 1e-5 over the whole UNMASKED tensor (quantise first, then
+ *             sparsify). The mean is exact and order-independent: every |w| is
+ *             truncated to a multiple of 2^-32, summed as an integer, and the sum /
+ *             (n * 2^32) is rounded once to fp32 (ties to even).
+ *   code    = RoundClip(w / gamma, -1, 1) (fp32 division, round half to even).
+ *   mask    = per group of m_group contiguous weights along k_in, keep the n_keep
+ *             largest |w| of the LATENT weights; equal |w| go to the lower index.
+ *   masked code = mask ? code : 0.
+ *
+ *   w_latent     [n_out, k_in] fp32, in.
+ *   n_keep, m_group: 1 <= n_keep <= m_group, m_group in {4, 8} (8:8 = no mask).
+ *   mask_out     [n_out, k_in / m_group] uint8, out, nullable. Bit j of byte g is
+ *                element j of group g (bits 0..3 only when m_group == 4).
+ *   codes_out    [n_out, k_in / 4] uint8, out. Masked codes, 4 per byte: element k
+ *                at bits 2*(k % 4) of byte k / 4; 00 = 0, 01 = +1, 11 = -1.
+ *   w_i8_out     [n_out, k_in] int8, out, nullable. Masked codes as int8 (the
+ *                operand of the tensor-core forward product).
+ *   w_scale_out  [1] fp32, out: gamma. NaN when the range check fails.
+ *   workspace    bitlinear_quant_mask_workspace_size() bytes, scratch, in/out.
+ *
+ * Range errors (non-finite w or |w| >= 2^16) are found on the device: gamma is then
+ * NaN, every code 0, and bitlinear_quant_mask_status() reports BL_ERR_RANGE.
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+bl_status bitlinear_quant_mask(const float* w_latent, int64_t n_out, int64_t k_in, int n_keep, int m_group,
+                               uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out, float* w_scale_out,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns the range status (BL_OK or BL_ERR_RANGE) that
+ * the last bitlinear_quant_mask using `workspace` recorded. */
+bl_status bitlinear_quant_mask_status(const void* workspace, void* stream);
+
+/*
+ * Step a3: per-token absmax int8 activation quantisation of X [t, k_in] (bf16).
+ *   a_t = max_k |x_tk|   (a zero row uses a_t = 1e-5, giving q = 0)
+ *   q   = clamp(rint(x * fp32(127 / a_t)), -128, 127), one fp32 multiply, ties to even.
+ *   xq_out [t, k_in] int8, out. absmax_out [t] fp32, out: a_t.
+ * Non-finite activations give unspecified (but in-bounds) results.
+ */
+bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t* xq_out, float* absmax_out,
+                              void* stream);
+
+/*
+ * Step a4: the masked ternary x int8 forward product.
+ *   acc[t, n] = sum_k xq[t, k] * masked_code[n, k]           (exact, int32)
+ *   y[t, n]   = acc * (absmax[t] / 127 * gamma)              (fp32, then bf16 or f32)
+ *
+ *   xq [t, k_in] int8, absmax [t] fp32 (from bitlinear_act_quant).
+ *   codes [n_out, k_in / 4] (packed masked codes), w_i8 [n_out, k_in] int8 (masked
+ *   codes): give at least one. With w_i8 the product runs on the tcgen05 int8 tensor
+ *   cores; with codes only it runs on a CUDA-core kernel that streams the 2-bit codes
+ *   (meant for short decode batches).
+ *   w_scale [1] fp32 gamma. acc_out [t, n_out] int32, out, nullable.
+ *   y_out [t, n_out], out, bf16 (y_dtype = BL_OUT_BF16) or fp32 (BL_OUT_F32).
+ * No bias term.
+ */
+bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* codes, const int8_t* w_i8,
+                        const float* w_scale, int64_t t, int64_t k_in, int64_t n_out, int32_t* acc_out, void* y_out,
+                        int y_dtype, void* stream);
+
+/* Bytes of workspace bitlinear_bwd needs (0 when grad_x is not requested). */
+size_t bitlinear_bwd_workspace_size(int64_t t, int64_t k_in, int64_t n_out, int want_grad_x);
+
+/*
+ * Steps a5 + a6: the dual straight-through backward.
+ *   grad_x[t, k] = sum_n dy[t, n] * gamma * masked_code[n, k]   (bf16 out, fp32 accumulate)
+ *   grad_w[n, k] = sum_t dy[t, n] * x[t, k]   for EVERY latent weight, masked ones
+ *                  included (the mask does not enter; fp32 accumulate).
+ *
+ *   dy [t, n_out] bf16, x [t, k_in] bf16 (the layer's bf16 input).
+ *   codes [n_out, k_in / 4] packed masked codes, w_scale [1] gamma (needed for grad_x).
+ *   grad_x [t, k_in] bf16, out, nullable. grad_w [n_out, k_in], out, nullable, bf16
+ *   (grad_w_dtype = BL_OUT_BF16) or fp32 (BL_OUT_F32). With t = 0, grad_w is zeroed.
+ *   workspace bitlinear_bwd_workspace_size() bytes (holds the bf16 ternary matrix).
+ */
+bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* codes, const float* w_scale, int64_t t,
+                        int64_t k_in, int64_t n_out, uint16_t* grad_x, void* grad_w, int grad_w_dtype,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises the current device, then returns BL_OK, or BL_ERR_TIMEOUT if a
+ * kernel of this library gave up on a bounded wait since the last call (the raw
+ * status bits go to *bits when bits != NULL). Clears the status. */
+bl_status bitlinear_device_status(unsigned int* bits);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+const char* bitlinear_last_error(void);
+
+/* ABI version of this header: 1. */
+int bitlinear_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

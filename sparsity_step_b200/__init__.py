@@ -1,1 +1,18 @@
-"""B200-native Sparse-BitNet BitLinear path (placeholder; binding added below)."""
+"""B200-native (sm_100a) Sparse-BitNet BitLinear path.
+
+The functions below are thin bindings of the C ABI in include/bitlinear.h; the
+library libbitlinear.so is loaded on first use and its absence is an error.
+"""
+from .bitlinear import (  # noqa: F401
+    BL_OUT_BF16,
+    BL_OUT_F32,
+    bitlinear_abi_version,
+    bitlinear_act_quant,
+    bitlinear_bwd,
+    bitlinear_bwd_workspace_size,
+    bitlinear_device_status,
+    bitlinear_fwd,
+    bitlinear_quant_mask,
+    bitlinear_quant_mask_status,
+    bitlinear_quant_mask_workspace_size,
+)

@@ -1,0 +1,157 @@
+"""Python binding of the BitLinear C ABI (include/bitlinear.h).
+
+Argument marshalling only: each function checks dtypes, devices and contiguity,
+allocates missing outputs with torch (device memory is PyTorch's job here), and
+passes raw pointers plus the current CUDA stream to the library. Every step of the
+computation runs in the library's CUDA kernels; there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import BL_OUT_BF16, BL_OUT_F32, check, lib
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def bitlinear_quant_mask_workspace_size(n_out: int, k_in: int) -> int:
+    return int(lib().bitlinear_quant_mask_workspace_size(n_out, k_in))
+
+
+def bitlinear_quant_mask(w: torch.Tensor, n_keep: int, m_group: int, *, want_mask: bool = True,
+                         want_w_i8: bool = True, out: dict | None = None, workspace: torch.Tensor | None = None,
+                         stream=None) -> dict:
+    """Mask, gamma and masked ternary codes of latent weights w [n_out, k_in] (fp32).
+
+    Returns a dict with ``codes`` (uint8 [n_out, k_in/4]), ``w_scale`` (fp32 [1]),
+    and optionally ``mask`` (uint8 [n_out, k_in/m]) and ``w_i8`` (int8 [n_out, k_in]).
+    """
+    n_out, k_in = w.shape
+    _need(w, torch.float32, None, "w")
+    dev = w.device
+    o = dict(out or {})
+    if "codes" not in o:
+        o["codes"] = torch.empty((n_out, k_in // 4), dtype=torch.uint8, device=dev)
+    if "w_scale" not in o:
+        o["w_scale"] = torch.empty((4,), dtype=torch.float32, device=dev)[:1]
+    if want_mask and "mask" not in o:
+        o["mask"] = torch.empty((n_out, k_in // m_group), dtype=torch.uint8, device=dev)
+    if want_w_i8 and "w_i8" not in o:
+        o["w_i8"] = torch.empty((n_out, k_in), dtype=torch.int8, device=dev)
+    ws_bytes = bitlinear_quant_mask_workspace_size(n_out, k_in)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    st = lib().bitlinear_quant_mask(_ptr(w), n_out, k_in, n_keep, m_group, _ptr(o.get("mask")), _ptr(o["codes"]),
+                                    _ptr(o.get("w_i8")), _ptr(o["w_scale"]), _ptr(workspace), workspace.numel(),
+                                    _stream(stream))
+    check(st, "bitlinear_quant_mask")
+    o["workspace"] = workspace
+    return o
+
+
+def bitlinear_quant_mask_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and return the range status (0 or BL_ERR_RANGE = -4); no raise."""
+    return int(lib().bitlinear_quant_mask_status(_ptr(workspace), _stream(stream)))
+
+
+def bitlinear_act_quant(x: torch.Tensor, *, xq: torch.Tensor | None = None, absmax: torch.Tensor | None = None,
+                        stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """int8 activations and per-token absmax of x [t, k_in] (bf16)."""
+    t, k_in = x.shape
+    _need(x, torch.bfloat16, None, "x")
+    if xq is None:
+        xq = torch.empty((t, k_in), dtype=torch.int8, device=x.device)
+    if absmax is None:
+        absmax = torch.empty((max(t, 1) + 3) // 4 * 4, dtype=torch.float32, device=x.device)[:t]
+    _need(xq, torch.int8, (t, k_in), "xq")
+    st = lib().bitlinear_act_quant(_ptr(x), t, k_in, _ptr(xq), _ptr(absmax), _stream(stream))
+    check(st, "bitlinear_act_quant")
+    return xq, absmax
+
+
+def bitlinear_fwd(xq: torch.Tensor, absmax: torch.Tensor, w_scale: torch.Tensor, *, codes: torch.Tensor | None = None,
+                  w_i8: torch.Tensor | None = None, n_out: int | None = None, y_dtype=torch.bfloat16,
+                  want_acc: bool = False, y: torch.Tensor | None = None, acc: torch.Tensor | None = None,
+                  stream=None) -> tuple[torch.Tensor, torch.Tensor | None]:
+    """y = (xq . masked_codes^T) * absmax/127 * gamma; returns (y, acc or None)."""
+    t, k_in = xq.shape
+    if n_out is None:
+        n_out = (w_i8 if w_i8 is not None else codes).shape[0]
+    if y is None:
+        y = torch.empty((t, n_out), dtype=y_dtype, device=xq.device)
+    if want_acc and acc is None:
+        acc = torch.empty((t, n_out), dtype=torch.int32, device=xq.device)
+    ydt = BL_OUT_F32 if y.dtype == torch.float32 else BL_OUT_BF16
+    st = lib().bitlinear_fwd(_ptr(xq), _ptr(absmax), _ptr(codes), _ptr(w_i8), _ptr(w_scale), t, k_in, n_out,
+                             _ptr(acc), _ptr(y), ydt, _stream(stream))
+    check(st, "bitlinear_fwd")
+    return y, acc
+
+
+def bitlinear_bwd_workspace_size(t: int, k_in: int, n_out: int, want_grad_x: bool = True) -> int:
+    return int(lib().bitlinear_bwd_workspace_size(t, k_in, n_out, int(want_grad_x)))
+
+
+def bitlinear_bwd(dy: torch.Tensor, x: torch.Tensor | None, codes: torch.Tensor | None, w_scale: torch.Tensor | None, *,
+                  want_grad_x: bool = True, want_grad_w: bool = True, grad_w_dtype=torch.bfloat16,
+                  grad_x: torch.Tensor | None = None, grad_w: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None, k_in: int | None = None,
+                  stream=None) -> tuple[torch.Tensor | None, torch.Tensor | None]:
+    """Dual straight-through backward; returns (grad_x or None, grad_w or None)."""
+    t, n_out = dy.shape
+    _need(dy, torch.bfloat16, None, "dy")
+    if k_in is None:
+        k_in = x.shape[1] if x is not None else codes.shape[1] * 4
+    dev = dy.device
+    if want_grad_x and grad_x is None:
+        grad_x = torch.empty((t, k_in), dtype=torch.bfloat16, device=dev)
+    if want_grad_w and grad_w is None:
+        grad_w = torch.empty((n_out, k_in), dtype=grad_w_dtype, device=dev)
+    gwdt = BL_OUT_F32 if (grad_w is not None and grad_w.dtype == torch.float32) else BL_OUT_BF16
+    need = bitlinear_bwd_workspace_size(t, k_in, n_out, grad_x is not None)
+    if need and workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    st = lib().bitlinear_bwd(_ptr(dy), _ptr(x), _ptr(codes), _ptr(w_scale), t, k_in, n_out, _ptr(grad_x), _ptr(grad_w),
+                             gwdt, _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
+    check(st, "bitlinear_bwd")
+    return grad_x, grad_w
+
+
+def bitlinear_device_status() -> tuple[int, int]:
+    """(status, bits): synchronise the device and read/clear the library's timeout bits."""
+    bits = ctypes.c_uint(0)
+    st = lib().bitlinear_device_status(ctypes.byref(bits))
+    return int(st), int(bits.value)
+
+
+def bitlinear_abi_version() -> int:
+    return int(lib().bitlinear_abi_version())
+
+
+__all__ = [
+    "bitlinear_quant_mask_workspace_size", "bitlinear_quant_mask", "bitlinear_quant_mask_status",
+    "bitlinear_act_quant", "bitlinear_fwd", "bitlinear_bwd_workspace_size", "bitlinear_bwd",
+    "bitlinear_device_status", "bitlinear_abi_version", "BL_OUT_BF16", "BL_OUT_F32", "_lib",
+]

@@ -1,0 +1,106 @@
+// Step a3: per-token absmax int8 activation quantisation, fused into one read.
+//
+// BitNet b1.58 2B4T article (lsdiaocha.cn), section 一: activations are quantised
+// to 8-bit integers; section 四: W1.58A8 (ternary weights x int8 activations).
+//
+// One CTA per token row. Each thread loads its 16-byte vectors of the row once and
+// keeps them in registers; the row absmax is a block max over |bf16| bit patterns
+// (exact, order-free); then q = clamp(rint(x * (127 / a)), -128, 127) with one
+// IEEE fp32 division per row and one fp32 multiply per element (no FMA), and the
+// int8 row is written with 8-byte stores. HBM traffic: 2 B read + 1 B written per
+// element, + 4 B per row.
+#pragma once
+
+#include "common.cuh"
+
+namespace bl {
+
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t w, uint32_t m) {
+  const uint32_t lo = w & 0x7fffu, hi = (w >> 16) & 0x7fffu;
+  return max(m, max(lo, hi));
+}
+
+__device__ __forceinline__ int quant_one(uint32_t bf16_bits, float s) {
+  const float xf = __uint_as_float(bf16_bits << 16);
+  const int q = __float2int_rn(__fmul_rn(xf, s));   // round half to even
+  return min(127, max(-128, q));
+}
+
+__device__ __forceinline__ uint32_t quant_pack4(uint32_t w0, uint32_t w1, float s) {
+  const int q0 = quant_one(w0 & 0xffffu, s), q1 = quant_one(w0 >> 16, s);
+  const int q2 = quant_one(w1 & 0xffffu, s), q3 = quant_one(w1 >> 16, s);
+  return (static_cast<uint32_t>(q0) & 0xffu) | ((static_cast<uint32_t>(q1) & 0xffu) << 8) |
+         ((static_cast<uint32_t>(q2) & 0xffu) << 16) | ((static_cast<uint32_t>(q3) & 0xffu) << 24);
+}
+
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t m, uint32_t* s_red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  uint32_t r = 0;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) r = max(r, s_red[w]);
+  return r;
+}
+
+// Row cached in registers: VPT 16-byte vectors (8 bf16 each) per thread.
+template <int VPT>
+__global__ void __launch_bounds__(256) act_quant_kernel(const uint4* __restrict__ x, int k8, int8_t* __restrict__ xq,
+                                                        float* __restrict__ absmax_out) {
+  __shared__ uint32_t s_red[8];
+  const int64_t row = blockIdx.x;
+  const uint4* xr = x + row * k8;
+  uint4 v[VPT];
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * blockDim.x;
+    if (idx < k8) {
+      v[i] = __ldcs(xr + idx);
+      m = bf16x2_absmax(v[i].x, m);
+      m = bf16x2_absmax(v[i].y, m);
+      m = bf16x2_absmax(v[i].z, m);
+      m = bf16x2_absmax(v[i].w, m);
+    }
+  }
+  m = block_max_u32(m, s_red);
+  float a = __uint_as_float(m << 16);
+  if (a == 0.0f) a = 1e-5f;   // an all-zero row quantises to zeros
+  const float s = __fdiv_rn(127.0f, a);
+  uint2* out = reinterpret_cast<uint2*>(xq + row * (static_cast<int64_t>(k8) * 8));
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * blockDim.x;
+    if (idx < k8) out[idx] = make_uint2(quant_pack4(v[i].x, v[i].y, s), quant_pack4(v[i].z, v[i].w, s));
+  }
+  if (threadIdx.x == 0) absmax_out[row] = a;
+}
+
+// Rows too long to cache in registers: read the row twice (max, then quantise).
+__global__ void __launch_bounds__(256) act_quant_long_kernel(const uint4* __restrict__ x, int k8, int8_t* __restrict__ xq,
+                                                             float* __restrict__ absmax_out) {
+  __shared__ uint32_t s_red[8];
+  const int64_t row = blockIdx.x;
+  const uint4* xr = x + row * k8;
+  uint32_t m = 0;
+  for (int idx = threadIdx.x; idx < k8; idx += blockDim.x) {
+    const uint4 v = xr[idx];
+    m = bf16x2_absmax(v.x, m);
+    m = bf16x2_absmax(v.y, m);
+    m = bf16x2_absmax(v.z, m);
+    m = bf16x2_absmax(v.w, m);
+  }
+  m = block_max_u32(m, s_red);
+  float a = __uint_as_float(m << 16);
+  if (a == 0.0f) a = 1e-5f;
+  const float s = __fdiv_rn(127.0f, a);
+  uint2* out = reinterpret_cast<uint2*>(xq + row * (static_cast<int64_t>(k8) * 8));
+  for (int idx = threadIdx.x; idx < k8; idx += blockDim.x) {
+    const uint4 v = __ldcs(xr + idx);
+    out[idx] = make_uint2(quant_pack4(v.x, v.y, s), quant_pack4(v.z, v.w, s));
+  }
+  if (threadIdx.x == 0) absmax_out[row] = a;
+}
+
+}  // namespace bl

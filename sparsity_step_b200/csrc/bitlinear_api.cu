@@ -1,0 +1,344 @@
+// C ABI of the BitLinear path (declared in include/bitlinear.h): argument checks,
+// workspace layout, TMA descriptor encoding and kernel dispatch. No allocation:
+// the caller owns every buffer.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/bitlinear.h"
+#include "act_quant.cuh"
+#include "codes_kernels.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "quant_mask.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+bl_status fail(bl_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bl_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+bl_status check_shape(int64_t t, int64_t k_in, int64_t n_out) {
+  if (t < 0 || t > (int64_t(1) << 31) - 1) return fail(BL_ERR_UNSUPPORTED_SHAPE, "t=%lld out of range", (long long)t);
+  if (k_in < 64 || k_in > 131072 || k_in % 64)
+    return fail(BL_ERR_UNSUPPORTED_SHAPE, "k_in=%lld: need 64 <= k_in <= 131072, k_in %% 64 == 0", (long long)k_in);
+  if (n_out < 16 || n_out % 16 || n_out > (int64_t(1) << 30))
+    return fail(BL_ERR_UNSUPPORTED_SHAPE, "n_out=%lld: need n_out >= 16, n_out %% 16 == 0", (long long)n_out);
+  return BL_OK;
+}
+
+int device_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 148;
+  return sms;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner], 128-byte swizzled boxes of [box_outer, box_inner].
+bl_status make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* base, uint64_t inner, uint64_t outer,
+                   uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(BL_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * elem};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return BL_OK;
+}
+
+template <bool kI8, bool kAMN, bool kBMN, int kEpi>
+bl_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const bl::GemmArgs& g, cudaStream_t st) {
+  auto kern = bl::gemm_tc_kernel<kI8, kAMN, kBMN, kEpi>;
+  static bool attr_set = false;   // per instantiation; cheap to repeat if raced
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bl::kGemmSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
+    attr_set = true;
+  }
+  const int tiles = g.num_m_blocks * g.num_n_blocks;
+  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  kern<<<grid, bl::kGemmThreads, bl::kGemmSmemBytes, st>>>(ta, tb, g);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return BL_OK;
+}
+
+// ------------------------------------------------------------------ quant_mask sizing
+
+constexpr int kQmTargetBlocks = 148 * 8;
+
+int qm_blocks(int64_t numel) {
+  const int64_t n4 = numel / 4;
+  int64_t need = (numel + (int64_t(bl::kQmThreads) * bl::kQmMaxElemsPerThread) - 1) /
+                 (int64_t(bl::kQmThreads) * bl::kQmMaxElemsPerThread);   // bounds elements per thread
+  int64_t fill = (n4 + bl::kQmThreads - 1) / bl::kQmThreads;
+  if (fill > kQmTargetBlocks) fill = kQmTargetBlocks;
+  int64_t b = need > fill ? need : fill;
+  if (b < 1) b = 1;
+  return static_cast<int>(b);
+}
+
+}  // namespace
+
+extern "C" {
+
+int bitlinear_abi_version(void) { return 1; }
+
+const char* bitlinear_last_error(void) { return g_err; }
+
+size_t bitlinear_quant_mask_workspace_size(int64_t n_out, int64_t k_in) {
+  if (n_out <= 0 || k_in <= 0) return bl::kQmWsHeader;
+  return bl::kQmWsHeader + 16 * static_cast<size_t>(qm_blocks(n_out * k_in));
+}
+
+bl_status bitlinear_quant_mask(const float* w_latent, int64_t n_out, int64_t k_in, int n_keep, int m_group,
+                               uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out, float* w_scale_out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  if (!w_latent || !codes_out || !w_scale_out) return fail(BL_ERR_INVALID_ARG, "w_latent, codes_out, w_scale_out are required");
+  if (bl_status s = check_shape(0, k_in, n_out)) return s;
+  if (!(m_group == 4 || m_group == 8) || n_keep < 1 || n_keep > m_group)
+    return fail(BL_ERR_INVALID_ARG, "N:M = %d:%d: need M in {4, 8} and 1 <= N <= M", n_keep, m_group);
+  if (!workspace) return fail(BL_ERR_WORKSPACE, "workspace is required");
+  const int64_t numel = n_out * k_in;
+  if (workspace_bytes < bitlinear_quant_mask_workspace_size(n_out, k_in))
+    return fail(BL_ERR_WORKSPACE, "workspace too small: %zu < %zu", workspace_bytes,
+                bitlinear_quant_mask_workspace_size(n_out, k_in));
+  if (!aligned16(w_latent) || !aligned16(codes_out) || !aligned16(w_scale_out) || !aligned16(workspace) ||
+      (mask_out && !aligned16(mask_out)) || (w_i8_out && !aligned16(w_i8_out)))
+    return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned int* range_flag = reinterpret_cast<unsigned int*>(ws);
+  int* status = reinterpret_cast<int*>(ws + 4);
+  unsigned long long* partials = reinterpret_cast<unsigned long long*>(ws + bl::kQmWsHeader);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 16, st);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
+  const int blocks = qm_blocks(numel);
+  bl::qm_abs_sum_kernel<<<blocks, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), numel / 4, partials,
+                                                          range_flag);
+  bl::qm_finalize_kernel<<<1, 256, 0, st>>>(partials, blocks, numel, range_flag, status, w_scale_out);
+  const int64_t n8 = numel / 8;
+  int64_t g2 = (n8 + bl::kQmThreads - 1) / bl::kQmThreads;
+  const int64_t cap = int64_t(device_sm_count()) * 16;
+  if (g2 > cap) g2 = cap;
+  if (m_group == 8)
+    bl::qm_mask_codes_kernel<8><<<(int)g2, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), n8, n_keep,
+                                                                     w_scale_out, mask_out,
+                                                                     reinterpret_cast<uint16_t*>(codes_out),
+                                                                     reinterpret_cast<uint2*>(w_i8_out));
+  else
+    bl::qm_mask_codes_kernel<4><<<(int)g2, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), n8, n_keep,
+                                                                     w_scale_out, mask_out,
+                                                                     reinterpret_cast<uint16_t*>(codes_out),
+                                                                     reinterpret_cast<uint2*>(w_i8_out));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quant_mask launch");
+  return BL_OK;
+}
+
+bl_status bitlinear_quant_mask_status(const void* workspace, void* stream) {
+  g_err[0] = 0;
+  if (!workspace) return fail(BL_ERR_WORKSPACE, "workspace is required");
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int status = 0;
+  e = cudaMemcpy(&status, static_cast<const uint8_t*>(workspace) + 4, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (status == BL_ERR_RANGE) return fail(BL_ERR_RANGE, "latent weight non-finite or |w| >= 2^16");
+  return BL_OK;
+}
+
+bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t* xq_out, float* absmax_out, void* stream) {
+  g_err[0] = 0;
+  if (!x || !xq_out || !absmax_out) return fail(BL_ERR_INVALID_ARG, "x, xq_out, absmax_out are required");
+  if (bl_status s = check_shape(t, k_in, 16)) return s;
+  if (!aligned16(x) || !aligned16(xq_out) || !aligned16(absmax_out))
+    return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  if (t == 0) return BL_OK;
+  cudaStream_t st = as_stream(stream);
+  const int k8 = static_cast<int>(k_in / 8);
+  const uint4* xv = reinterpret_cast<const uint4*>(x);
+  const unsigned grid = static_cast<unsigned>(t);
+  if (k8 <= 128) {
+    bl::act_quant_kernel<1><<<grid, 128, 0, st>>>(xv, k8, xq_out, absmax_out);
+  } else {
+    const int vpt = (k8 + 255) / 256;
+    if (vpt <= 2) bl::act_quant_kernel<2><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+    else if (vpt <= 4) bl::act_quant_kernel<4><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+    else if (vpt <= 6) bl::act_quant_kernel<6><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+    else if (vpt <= 8) bl::act_quant_kernel<8><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+    else if (vpt <= 12) bl::act_quant_kernel<12><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+    else if (vpt <= 16) bl::act_quant_kernel<16><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+    else bl::act_quant_long_kernel<<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  return BL_OK;
+}
+
+bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* codes, const int8_t* w_i8,
+                        const float* w_scale, int64_t t, int64_t k_in, int64_t n_out, int32_t* acc_out, void* y_out,
+                        int y_dtype, void* stream) {
+  g_err[0] = 0;
+  if (!xq || !absmax || !w_scale || !y_out) return fail(BL_ERR_INVALID_ARG, "xq, absmax, w_scale, y_out are required");
+  if (!codes && !w_i8) return fail(BL_ERR_INVALID_ARG, "give codes or w_i8");
+  if (y_dtype != BL_OUT_BF16 && y_dtype != BL_OUT_F32) return fail(BL_ERR_INVALID_ARG, "y_dtype must be BL_OUT_BF16 or BL_OUT_F32");
+  if (bl_status s = check_shape(t, k_in, n_out)) return s;
+  if (!aligned16(xq) || !aligned16(absmax) || !aligned16(w_scale) || !aligned16(y_out) || (codes && !aligned16(codes)) ||
+      (w_i8 && !aligned16(w_i8)) || (acc_out && !aligned16(acc_out)))
+    return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  if (t == 0) return BL_OK;
+  cudaStream_t st = as_stream(stream);
+  if (w_i8) {
+    CUtensorMap ta, tb;
+    if (bl_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, k_in, t, 128, bl::kBM)) return s;
+    if (bl_status s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_i8, k_in, n_out, 128, bl::kBN)) return s;
+    bl::GemmArgs g{};
+    g.M = static_cast<int>(t);
+    g.N = static_cast<int>(n_out);
+    g.num_k_blocks = static_cast<int>((k_in + 127) / 128);
+    g.num_m_blocks = static_cast<int>((t + bl::kBM - 1) / bl::kBM);
+    g.num_n_blocks = static_cast<int>((n_out + bl::kBN - 1) / bl::kBN);
+    g.out = y_out;
+    g.out_f32 = y_dtype == BL_OUT_F32;
+    g.acc_out = acc_out;
+    g.row_absmax = absmax;
+    g.w_scale = w_scale;
+    return launch_gemm<true, false, false, bl::EPI_FWD>(ta, tb, g, st);
+  }
+  const unsigned grid = static_cast<unsigned>((n_out + bl::kCodesWarps - 1) / bl::kCodesWarps);
+  bl::fwd_codes_kernel<<<grid, bl::kCodesWarps * 32, 0, st>>>(xq, absmax, codes, w_scale, static_cast<int>(t),
+                                                              static_cast<int>(k_in), static_cast<int>(n_out), acc_out,
+                                                              y_out, y_dtype == BL_OUT_F32);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fwd_codes launch");
+  return BL_OK;
+}
+
+size_t bitlinear_bwd_workspace_size(int64_t t, int64_t k_in, int64_t n_out, int want_grad_x) {
+  (void)t;
+  if (!want_grad_x || k_in <= 0 || n_out <= 0) return 0;
+  return static_cast<size_t>(n_out) * static_cast<size_t>(k_in) * 2;
+}
+
+bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* codes, const float* w_scale, int64_t t,
+                        int64_t k_in, int64_t n_out, uint16_t* grad_x, void* grad_w, int grad_w_dtype, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  if (!grad_x && !grad_w) return fail(BL_ERR_INVALID_ARG, "request grad_x, grad_w or both");
+  if (!dy) return fail(BL_ERR_INVALID_ARG, "dy is required");
+  if (grad_x && (!codes || !w_scale)) return fail(BL_ERR_INVALID_ARG, "grad_x needs codes and w_scale");
+  if (grad_w && !x) return fail(BL_ERR_INVALID_ARG, "grad_w needs x");
+  if (grad_w && grad_w_dtype != BL_OUT_BF16 && grad_w_dtype != BL_OUT_F32)
+    return fail(BL_ERR_INVALID_ARG, "grad_w_dtype must be BL_OUT_BF16 or BL_OUT_F32");
+  if (bl_status s = check_shape(t, k_in, n_out)) return s;
+  if (!aligned16(dy) || (x && !aligned16(x)) || (codes && !aligned16(codes)) || (w_scale && !aligned16(w_scale)) ||
+      (grad_x && !aligned16(grad_x)) || (grad_w && !aligned16(grad_w)) || (workspace && !aligned16(workspace)))
+    return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  const size_t need = bitlinear_bwd_workspace_size(t, k_in, n_out, grad_x != nullptr);
+  if (need && (!workspace || workspace_bytes < need))
+    return fail(BL_ERR_WORKSPACE, "workspace too small: %zu < %zu", workspace_bytes, need);
+  cudaStream_t st = as_stream(stream);
+  if (t == 0) {
+    if (grad_w) {
+      const size_t bytes = static_cast<size_t>(n_out) * k_in * (grad_w_dtype == BL_OUT_F32 ? 4 : 2);
+      cudaError_t e = cudaMemsetAsync(grad_w, 0, bytes, st);
+      if (e != cudaSuccess) return cuda_fail(e, "grad_w zero");
+    }
+    return BL_OK;
+  }
+  if (grad_x) {
+    // effective ternary matrix C [n_out, k_in] in bf16 (exact), gamma applied in the epilogue
+    const int64_t nwords = n_out * k_in / 16;
+    int64_t grid = (nwords + 255) / 256;
+    const int64_t cap = int64_t(device_sm_count()) * 16;
+    if (grid > cap) grid = cap;
+    bl::expand_codes_bf16_kernel<<<(int)grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(codes), nwords,
+                                                           static_cast<uint4*>(workspace));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "expand launch");
+    CUtensorMap ta, tb;
+    // A = dY [t, n_out], K-major (reduction over n_out); B = C [n_out, k_in], MN-major
+    if (bl_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dy, n_out, t, 64, bl::kBM)) return s;
+    if (bl_status s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, workspace, k_in, n_out, 64, 64)) return s;
+    bl::GemmArgs g{};
+    g.M = static_cast<int>(t);
+    g.N = static_cast<int>(k_in);
+    g.num_k_blocks = static_cast<int>((n_out + 63) / 64);
+    g.num_m_blocks = static_cast<int>((t + bl::kBM - 1) / bl::kBM);
+    g.num_n_blocks = static_cast<int>((k_in + bl::kBN - 1) / bl::kBN);
+    g.out = grad_x;
+    g.out_f32 = 0;
+    g.w_scale = w_scale;
+    if (bl_status s = launch_gemm<false, false, true, bl::EPI_GRADX>(ta, tb, g, st)) return s;
+  }
+  if (grad_w) {
+    CUtensorMap ta, tb;
+    // A = dY^T: dY [t, n_out] read MN-major (reduction over t); B = X [t, k_in], MN-major
+    if (bl_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dy, n_out, t, 64, 64)) return s;
+    if (bl_status s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, k_in, t, 64, 64)) return s;
+    bl::GemmArgs g{};
+    g.M = static_cast<int>(n_out);
+    g.N = static_cast<int>(k_in);
+    g.num_k_blocks = static_cast<int>((t + 63) / 64);
+    g.num_m_blocks = static_cast<int>((n_out + bl::kBM - 1) / bl::kBM);
+    g.num_n_blocks = static_cast<int>((k_in + bl::kBN - 1) / bl::kBN);
+    g.out = grad_w;
+    g.out_f32 = grad_w_dtype == BL_OUT_F32;
+    if (bl_status s = launch_gemm<false, true, true, bl::EPI_GRADW>(ta, tb, g, st)) return s;
+  }
+  return BL_OK;
+}
+
+bl_status bitlinear_device_status(unsigned int* bits) {
+  g_err[0] = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "device synchronize");
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, bl::g_device_status, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  e = cudaMemcpyToSymbol(bl::g_device_status, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  if (bits) *bits = v;
+  if (v) return fail(BL_ERR_TIMEOUT, "a kernel gave up on a bounded wait (status bits 0x%x)", v);
+  return BL_OK;
+}
+
+}  // extern "C"

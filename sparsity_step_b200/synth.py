@@ -20,6 +20,9 @@ Generator (stated so that anyone can re-implement it bit for bit):
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 _GOLDEN = np.uint64(0x9E3779B97F4A7C15)
@@ -51,26 +54,36 @@ def uniform01(seed: int, salt: int, start: int, count: int) -> np.ndarray:
     return (z >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
 
 
+def _chunked(count: int, fill) -> np.ndarray:
+    """Fill an fp64 array chunk by chunk; chunks are independent (counter-based
+    streams), so they run on a thread pool without changing any value."""
+    out = np.empty(count, dtype=np.float64)
+    starts = list(range(0, count, _CHUNK))
+    if len(starts) <= 1:
+        for s in starts:
+            fill(out, s, min(_CHUNK, count - s))
+        return out
+    with ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 1)) as ex:
+        list(ex.map(lambda s: fill(out, s, min(_CHUNK, count - s)), starts))
+    return out
+
+
 def normal_f64(seed: int, count: int, std: float = 1.0) -> np.ndarray:
     """``count`` iid N(0, std^2) samples in fp64 (std is the standard deviation)."""
-    out = np.empty(count, dtype=np.float64)
-    for s in range(0, count, _CHUNK):
-        c = min(_CHUNK, count - s)
+    def fill(out, s, c):
         z = splitmix64(seed, SALT_NORMAL, 2 * s, 2 * c)
         u1 = ((z[0::2] >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
         u2 = (z[1::2] >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
         out[s:s + c] = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2) * std
-    return out
+    return _chunked(count, fill)
 
 
 def outlier_factor(seed: int, count: int, p: float = 0.01, scale: float = 20.0) -> np.ndarray:
     """Per-element factor: ``scale`` with probability ``p``, else 1."""
-    out = np.empty(count, dtype=np.float64)
-    for s in range(0, count, _CHUNK):
-        c = min(_CHUNK, count - s)
+    def fill(out, s, c):
         u = uniform01(seed, SALT_OUTLIER, s, c)
         out[s:s + c] = np.where(u < p, scale, 1.0)
-    return out
+    return _chunked(count, fill)
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:

@@ -1,0 +1,113 @@
+"""The C-ABI library builds, loads and exports every declared symbol; host-side
+argument validation rejects bad calls before anything is enqueued (CPU only: no
+call here reaches a CUDA API)."""
+import ctypes
+
+import pytest
+
+from sparsity_step_b200 import _lib
+from sparsity_step_b200.build import build
+
+BAD = 0x1001          # a misaligned fake device address (never dereferenced)
+GOOD = 0x10000        # an aligned fake device address (never dereferenced)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _lib.lib()
+
+
+def test_exports_every_header_function(L):
+    names = _lib.header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+def test_abi_version(L):
+    assert L.bitlinear_abi_version() == 1
+
+
+def _err(L):
+    return L.bitlinear_last_error().decode()
+
+
+def test_quant_mask_validation(L):
+    ws = L.bitlinear_quant_mask_workspace_size(896, 896)
+    assert ws >= 256 + 16
+    # null latent weights
+    assert L.bitlinear_quant_mask(None, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -1
+    # bad N:M
+    for n, m in [(0, 8), (9, 8), (2, 3), (6, 16)]:
+        assert L.bitlinear_quant_mask(GOOD, 896, 896, n, m, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -1
+    # unsupported shapes
+    assert L.bitlinear_quant_mask(GOOD, 896, 900, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -2
+    assert L.bitlinear_quant_mask(GOOD, 8, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -2
+    # workspace
+    assert L.bitlinear_quant_mask(GOOD, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, None, ws, None) == -7
+    assert L.bitlinear_quant_mask(GOOD, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws - 1, None) == -7
+    # alignment
+    assert L.bitlinear_quant_mask(BAD, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -3
+    assert "aligned" in _err(L)
+
+
+def test_act_quant_validation(L):
+    assert L.bitlinear_act_quant(None, 4, 896, GOOD, GOOD, None) == -1
+    assert L.bitlinear_act_quant(GOOD, 4, 100, GOOD, GOOD, None) == -2
+    assert L.bitlinear_act_quant(GOOD, -1, 896, GOOD, GOOD, None) == -2
+    assert L.bitlinear_act_quant(GOOD, 4, 896, BAD, GOOD, None) == -3
+    # an empty batch is valid and enqueues nothing
+    assert L.bitlinear_act_quant(GOOD, 0, 896, GOOD, GOOD, None) == 0
+
+
+def test_fwd_validation(L):
+    args = dict(xq=GOOD, a=GOOD, codes=GOOD, wi8=GOOD, g=GOOD)
+    assert L.bitlinear_fwd(GOOD, GOOD, None, None, GOOD, 4, 896, 896, None, GOOD, 0, None) == -1
+    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, GOOD, 4, 896, 896, None, GOOD, 7, None) == -1
+    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, GOOD, 4, 896, 100, None, GOOD, 0, None) == -2
+    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, GOOD, 4, 896, 896, BAD, GOOD, 0, None) == -3
+    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, GOOD, 0, 896, 896, None, GOOD, 0, None) == 0
+    del args
+
+
+def test_bwd_validation(L):
+    need = L.bitlinear_bwd_workspace_size(16, 896, 896, 1)
+    assert need == 896 * 896 * 2
+    assert L.bitlinear_bwd_workspace_size(16, 896, 896, 0) == 0
+    # nothing requested
+    assert L.bitlinear_bwd(GOOD, GOOD, GOOD, GOOD, 16, 896, 896, None, None, 0, GOOD, need, None) == -1
+    # grad_x without codes
+    assert L.bitlinear_bwd(GOOD, GOOD, None, GOOD, 16, 896, 896, GOOD, None, 0, GOOD, need, None) == -1
+    # workspace too small for grad_x
+    assert L.bitlinear_bwd(GOOD, GOOD, GOOD, GOOD, 16, 896, 896, GOOD, None, 0, GOOD, need - 16, None) == -7
+    # grad_w only needs no workspace; bad dtype is rejected
+    assert L.bitlinear_bwd(GOOD, GOOD, None, None, 16, 896, 896, None, GOOD, 3, None, 0, None) == -1
+    assert L.bitlinear_bwd(GOOD, BAD, None, None, 16, 896, 896, None, GOOD, 0, None, 0, None) == -3
+
+
+def test_last_error_is_thread_local_message(L):
+    assert L.bitlinear_act_quant(None, 4, 896, GOOD, GOOD, None) == -1
+    assert "required" in _err(L)
+    assert L.bitlinear_act_quant(GOOD, 0, 896, GOOD, GOOD, None) == 0
+    assert _err(L) == ""
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_LIB", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        _lib.lib()
+
+
+def test_ctypes_signatures_match_header_arity():
+    import re
+    with open(_lib.HEADER) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    for name, (_, args) in _lib.SIGNATURES.items():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", text)
+        assert m, name
+        params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        assert len(params) == len(args), name
+    assert ctypes.sizeof(ctypes.c_size_t) == 8

@@ -1,0 +1,261 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, on seeded
+inputs of every workload shape (full outputs where the oracle is quick, sampled
+rows at full launch sizes) and on the edge cases of the method."""
+import numpy as np
+import pytest
+import torch
+
+import sparsity_step_b200 as B
+from oracle import bitlinear_oracle as O
+from parity_util import (assert_bf16_within_ulp, assert_exact, assert_f32_close, assert_grad_close, bf16_dev_to_bits,
+                         bits_to_dev_bf16, f32_to_dev, layer_inputs, sample_rows)
+from sparsity_step_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+# ------------------------------------------------------------------ shared checks
+
+
+def gpu_quant_mask(w_np, n, m):
+    out = B.bitlinear_quant_mask(f32_to_dev(w_np), n, m)
+    torch.cuda.synchronize()
+    assert B.bitlinear_quant_mask_status(out["workspace"]) == 0
+    return out
+
+
+def check_quant_mask(out, ref, tag):
+    g = out["w_scale"].cpu().numpy()[:1]
+    assert_exact(g.view(np.uint32), np.array([ref["gamma"]], np.float32).view(np.uint32), f"{tag} gamma")
+    assert_exact(out["mask"].cpu().numpy(), ref["mask"], f"{tag} mask")
+    assert_exact(out["codes"].cpu().numpy(), ref["codes_packed"], f"{tag} codes")
+    assert_exact(out["w_i8"].cpu().numpy(), ref["mcode"], f"{tag} w_i8")
+
+
+def gpu_act_quant(x_bits):
+    xq, a = B.bitlinear_act_quant(bits_to_dev_bf16(x_bits))
+    torch.cuda.synchronize()
+    return xq, a
+
+
+def check_act_quant(xq, a, ref_q, ref_a, tag):
+    assert_exact(xq.cpu().numpy(), ref_q, f"{tag} xq")
+    assert_exact(a.cpu().numpy().view(np.uint32), ref_a.astype(np.float32).view(np.uint32), f"{tag} absmax")
+
+
+def check_fwd(qm_dev, xq, a, ref_qm, ref_q, ref_a, tag, rows=None, paths=("w_i8",), f32=True):
+    """Forward on both requested weight operands; compares acc (exact), bf16 and f32 y."""
+    acc_ref, y_ref = O.fwd(ref_q, ref_a, ref_qm["mcode"], ref_qm["gamma"], rows=rows)
+    for path in paths:
+        kw = {"w_i8": qm_dev["w_i8"]} if path == "w_i8" else {"codes": qm_dev["codes"]}
+        y, acc = B.bitlinear_fwd(xq, a, qm_dev["w_scale"], n_out=ref_qm["mcode"].shape[0], want_acc=True, **kw)
+        torch.cuda.synchronize()
+        acc_np = acc.cpu().numpy()
+        ybits = bf16_dev_to_bits(y)
+        if rows is not None:
+            acc_np, ybits = acc_np[rows], ybits[rows]
+        assert_exact(acc_np, acc_ref, f"{tag} acc [{path}]")
+        assert_bf16_within_ulp(ybits, y_ref, f"{tag} y bf16 [{path}]")
+        if f32:
+            y32, _ = B.bitlinear_fwd(xq, a, qm_dev["w_scale"], n_out=ref_qm["mcode"].shape[0], y_dtype=torch.float32, **kw)
+            torch.cuda.synchronize()
+            y32 = y32.cpu().numpy()
+            if rows is not None:
+                y32 = y32[rows]
+            assert_f32_close(y32, y_ref, f"{tag} y f32 [{path}]")
+
+
+def check_bwd(dy_bits, x_bits, qm_dev, ref_qm, tag, rows_t=None, rows_n=None, gw_f32=False):
+    dy = bits_to_dev_bf16(dy_bits)
+    x = bits_to_dev_bf16(x_bits)
+    gx, gw = B.bitlinear_bwd(dy, x, qm_dev["codes"], qm_dev["w_scale"],
+                             grad_w_dtype=torch.float32 if gw_f32 else torch.bfloat16)
+    torch.cuda.synchronize()
+    gx_ref = O.grad_x(dy_bits, ref_qm["mcode"], ref_qm["gamma"], rows=rows_t)
+    gw_ref = O.grad_w(dy_bits, x_bits, rows=rows_n)
+    gxb = bf16_dev_to_bits(gx)
+    assert_grad_close(gxb if rows_t is None else gxb[rows_t], gx_ref, f"{tag} grad_x")
+    if gw_f32:
+        g = gw.cpu().numpy()
+        assert_grad_close(g if rows_n is None else g[rows_n], gw_ref, f"{tag} grad_w f32", is_bf16=False)
+    else:
+        g = bf16_dev_to_bits(gw)
+        assert_grad_close(g if rows_n is None else g[rows_n], gw_ref, f"{tag} grad_w")
+
+
+def full_layer(cfg, tensor, t, k_in, n_out, n, m, *, outliers=True, bwd=True, paths=("w_i8", "codes"), sample=False):
+    w, x, dy = layer_inputs(cfg, tensor, t, k_in, n_out, outliers=outliers)
+    tag = f"cfg{cfg} t{tensor} [{t}x{k_in}->{n_out}] {n}:{m}"
+    ref_qm = O.quant_mask(w, n, m)
+    qm = gpu_quant_mask(w, n, m)
+    check_quant_mask(qm, ref_qm, tag)
+    ref_q, ref_a = O.act_quant(x)
+    xq, a = gpu_act_quant(x)
+    check_act_quant(xq, a, ref_q, ref_a, tag)
+    rows = sample_rows(t, tensor) if sample else None
+    check_fwd(qm, xq, a, ref_qm, ref_q, ref_a, tag, rows=rows, paths=paths)
+    if bwd:
+        check_bwd(dy, x, qm, ref_qm, tag, rows_t=rows, rows_n=sample_rows(n_out, tensor + 7) if sample else None)
+
+
+# ------------------------------------------------------------------ the five workloads
+
+
+def test_config1_single_layer_full():
+    """X 64x896 bf16 N(0,1) + 1% x20, W 896x896 N(0,0.02), 6:8, seed 0: every output."""
+    full_layer(1, 0, 64, 896, 896, 6, 8)
+
+
+QWEN05 = [("q", 896, 896), ("k", 896, 128), ("v", 896, 128), ("o", 896, 896),
+          ("gate", 896, 4864), ("up", 896, 4864), ("down", 4864, 896)]
+
+
+@pytest.mark.parametrize("idx", range(len(QWEN05)), ids=[s[0] for s in QWEN05])
+def test_config2_qwen05_linears(idx):
+    _, k_in, n_out = QWEN05[idx]
+    full_layer(2, idx, 4096, k_in, n_out, 6, 8, bwd=False, paths=("w_i8",))
+
+
+QWEN15_MLP = [("gate", 1536, 8960), ("up", 1536, 8960), ("down", 8960, 1536)]
+
+
+@pytest.mark.parametrize("nm", [(8, 8), (6, 8), (4, 8), (2, 4), (2, 8)], ids=lambda v: f"{v[0]}of{v[1]}")
+@pytest.mark.parametrize("idx", range(3), ids=[s[0] for s in QWEN15_MLP])
+def test_config3_nm_sweep(idx, nm):
+    _, k_in, n_out = QWEN15_MLP[idx]
+    full_layer(3, idx, 8192, k_in, n_out, nm[0], nm[1], outliers=False, bwd=False, paths=("w_i8",), sample=True)
+
+
+QWEN3B_MLP = [("gate", 2048, 11008), ("up", 2048, 11008), ("down", 11008, 2048)]
+
+
+@pytest.mark.parametrize("idx", range(3), ids=[s[0] for s in QWEN3B_MLP])
+def test_config4_training_step(idx):
+    _, k_in, n_out = QWEN3B_MLP[idx]
+    full_layer(4, idx, 16384, k_in, n_out, 6, 8, bwd=True, paths=("w_i8",), sample=True)
+
+
+QWEN3B_LAYER = [("q", 2048, 2048), ("k", 2048, 256), ("v", 2048, 256), ("o", 2048, 2048),
+                ("gate", 2048, 11008), ("up", 2048, 11008), ("down", 11008, 2048)]
+
+
+@pytest.mark.parametrize("layer", [0, 35])
+@pytest.mark.parametrize("idx", range(len(QWEN3B_LAYER)), ids=[s[0] for s in QWEN3B_LAYER])
+def test_config5_decode_batches(idx, layer):
+    _, k_in, n_out = QWEN3B_LAYER[idx]
+    w = synth.latent_weight(synth.config_seed(5, 100 * layer + idx), n_out, k_in)
+    ref_qm = O.quant_mask(w, 6, 8)
+    qm = gpu_quant_mask(w, 6, 8)
+    check_quant_mask(qm, ref_qm, f"cfg5 L{layer} {QWEN3B_LAYER[idx][0]}")
+    for b in (1, 8, 32, 128):
+        x = synth.activation_bf16(synth.config_seed(5, 5000 + 10 * idx + b), b, k_in, outliers=False)
+        ref_q, ref_a = O.act_quant(x)
+        xq, a = gpu_act_quant(x)
+        check_act_quant(xq, a, ref_q, ref_a, f"cfg5 b{b}")
+        check_fwd(qm, xq, a, ref_qm, ref_q, ref_a, f"cfg5 L{layer} {QWEN3B_LAYER[idx][0]} b{b}", paths=("w_i8", "codes"),
+                  f32=(b == 8))
+
+
+@pytest.mark.parametrize("idx", [0, 6], ids=["q", "down"])
+def test_config5_prefill_8192(idx):
+    _, k_in, n_out = QWEN3B_LAYER[idx]
+    w = synth.latent_weight(synth.config_seed(5, idx), n_out, k_in)
+    x = synth.activation_bf16(synth.config_seed(5, 7000 + idx), 8192, k_in, outliers=False)
+    ref_qm = O.quant_mask(w, 6, 8)
+    qm = gpu_quant_mask(w, 6, 8)
+    ref_q, ref_a = O.act_quant(x)
+    xq, a = gpu_act_quant(x)
+    check_act_quant(xq, a, ref_q, ref_a, "cfg5 prefill")
+    check_fwd(qm, xq, a, ref_qm, ref_q, ref_a, "cfg5 prefill", rows=sample_rows(8192, idx), paths=("w_i8",), f32=False)
+
+
+# ------------------------------------------------------------------ edge cases
+
+
+@pytest.mark.parametrize("t", [1, 5, 127, 129, 300])
+def test_ragged_token_counts(t):
+    # k_in = 576 ends the int8 K loop on a half-filled 128-byte stage; n_out = 144
+    # ends the bf16 reduction of grad_x on a partial 64-row stage and leaves a
+    # ragged last tile in every product.
+    full_layer(1, 10 + t, t, 576, 144, 6, 8)
+
+
+@pytest.mark.parametrize("nm", [(6, 8), (4, 8), (3, 8), (2, 4), (1, 4), (8, 8)])
+def test_mask_ties(nm):
+    n, m = nm
+    rng = np.random.default_rng(3)
+    mag = rng.integers(0, 4, size=(64, 256)).astype(np.float32) * np.float32(0.01)
+    w = (mag * np.where(rng.random((64, 256)) < 0.5, -1, 1)).astype(np.float32)
+    w[0, :8] = 0.0   # an all-zero group (all ties, gamma still positive)
+    ref = O.quant_mask(w, n, m)
+    check_quant_mask(gpu_quant_mask(w, n, m), ref, f"ties {n}:{m}")
+
+
+def test_codes_at_rounding_boundary():
+    # weights at exactly +-gamma/2 (ties: code 0), one float above (code +-1), and 1.5 gamma
+    w = synth.latent_weight(77, 32, 64)
+    g, _, _ = O.absmean_gamma(w)
+    half = np.float32(0.5) * np.float32(g)
+    qm0 = O.quant_mask(w, 8, 8)
+    assert qm0["gamma"] == g
+    w2 = w.copy()
+    w2[0, 0], w2[0, 1] = half, -half
+    w2[0, 2] = np.nextafter(half, np.float32(1))
+    w2[0, 3] = np.float32(1.5) * np.float32(g)
+    ref = O.quant_mask(w2, 8, 8)
+    check_quant_mask(gpu_quant_mask(w2, 8, 8), ref, "boundary")
+
+
+def test_zero_activation_rows_and_empty_batch():
+    x = synth.activation_bf16(88, 6, 896)
+    x[2, :] = 0
+    ref_q, ref_a = O.act_quant(x)
+    xq, a = gpu_act_quant(x)
+    check_act_quant(xq, a, ref_q, ref_a, "zero row")
+    # empty batch: every entry point accepts t = 0; grad_w of an empty batch is zero
+    w = synth.latent_weight(89, 128, 896)
+    qm = gpu_quant_mask(w, 6, 8)
+    x0 = torch.empty((0, 896), dtype=torch.bfloat16, device="cuda")
+    xq0, a0 = B.bitlinear_act_quant(x0)
+    y0, _ = B.bitlinear_fwd(xq0, a0, qm["w_scale"], w_i8=qm["w_i8"])
+    assert y0.shape == (0, 128)
+    dy0 = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    gw = torch.full((128, 896), 7.0, dtype=torch.bfloat16, device="cuda")
+    B.bitlinear_bwd(dy0, x0, qm["codes"], qm["w_scale"], grad_w=gw)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(gw).item() == 0
+
+
+def test_grad_w_f32_and_masked_positions():
+    w, x, dy = layer_inputs(1, 40, 200, 896, 256)
+    ref_qm = O.quant_mask(w, 2, 8)
+    qm = gpu_quant_mask(w, 2, 8)
+    check_bwd(dy, x, qm, ref_qm, "gw f32", gw_f32=True)
+    # the straight-through gradient reaches masked weights: the GPU grad_W is the
+    # same for 2:8 and 8:8 masks
+    qm8 = gpu_quant_mask(w, 8, 8)
+    _, g2 = B.bitlinear_bwd(bits_to_dev_bf16(dy), bits_to_dev_bf16(x), qm["codes"], qm["w_scale"], want_grad_x=False)
+    _, g8 = B.bitlinear_bwd(bits_to_dev_bf16(dy), bits_to_dev_bf16(x), qm8["codes"], qm8["w_scale"], want_grad_x=False)
+    torch.cuda.synchronize()
+    assert torch.equal(g2, g8)
+
+
+def test_range_error_reported():
+    w = synth.latent_weight(90, 64, 128)
+    w[3, 5] = np.nan
+    out = B.bitlinear_quant_mask(f32_to_dev(w), 6, 8)
+    assert B.bitlinear_quant_mask_status(out["workspace"]) == -4
+    assert np.isnan(out["w_scale"].cpu().numpy()[0])
+    assert int(out["codes"].cpu().numpy().sum()) == 0
+    w[3, 5] = 70000.0
+    out = B.bitlinear_quant_mask(f32_to_dev(w), 6, 8, workspace=out["workspace"])
+    assert B.bitlinear_quant_mask_status(out["workspace"]) == -4
+    # the same workspace works again for valid weights
+    w[3, 5] = 0.01
+    out = B.bitlinear_quant_mask(f32_to_dev(w), 6, 8, workspace=out["workspace"])
+    assert B.bitlinear_quant_mask_status(out["workspace"]) == 0
+    check_quant_mask(out, O.quant_mask(w, 6, 8), "after range error")
+
+
+def test_no_device_timeouts():
+    st, bits = B.bitlinear_device_status()
+    assert st == 0 and bits == 0
