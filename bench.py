@@ -1,0 +1,504 @@
+"""Benchmark of the Sparse-BitNet BitLinear path on B200.
+
+One step = one pass of the whole path over one batch: for each linear of a
+Qwen2.5-3B-shaped MLP (gate 2048->11008, up 2048->11008, down 11008->2048) at
+16384 tokens and a 6:8 mask: recompute mask + ternary codes from the latent fp32
+weights, quantise the activations to int8, run the forward product, and both
+straight-through gradients (grad_X and grad_W over every latent weight).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). ``value`` is tokens per second of the whole job
+(all ranks; each rank runs its own batch: weak scaling, no collective on the data
+path). ``e2e`` is the same metric through the public API with the step's inputs
+copied from pinned host memory and its outputs copied back inside the timed region.
+``--impl reference`` times the CPU oracle (the slow reference implementation) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "6:8 ternary BitLinear TOPS & tok/s (fwd/bwd), % roofline, speedup vs 8:8 dense"
+WORKLOAD = "train-step Qwen2.5-3B MLP BitLinear (gate/up 2048->11008, down 11008->2048), 16384 tokens, 6:8"
+TOKENS = 16384
+LINEARS = [("gate", 2048, 11008), ("up", 2048, 11008), ("down", 11008, 2048)]
+N_KEEP, M_GROUP = 6, 8
+CFG_INDEX = 4   # the training-step workload's seed block
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture, keyed by the
+# SHA-256 of the kernel's source files at capture time (reported as null once the
+# source has changed).
+TRAFFIC = {}
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "sparsity_step_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    def __init__(self, gpu: str):
+        self.gpu = gpu   # nvidia-smi id: the device UUID (CUDA_VISIBLE_DEVICES does not apply there)
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.remove(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i - 5] for r in rows for i in range(5, 9) if r[i].lower().startswith("active")})
+        loaded = [s for s in sm if s >= 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
+
+
+def gpu_smi_id(local: int) -> str:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(local).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(local)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def make_inputs(rank: int):
+    import numpy as np
+    import torch
+
+    from sparsity_step_b200 import synth
+
+    off = 100000 * rank
+    host = {}
+    for i, (name, k_in, n_out) in enumerate(LINEARS):
+        host[f"w_{name}"] = synth.latent_weight(synth.config_seed(CFG_INDEX, 3 * i) + off, n_out, k_in)
+        host[f"dy_{name}"] = synth.activation_bf16(synth.config_seed(CFG_INDEX, 3 * i + 2) + off, TOKENS, n_out,
+                                                   std=1e-2, outliers=False)
+    host["x_in"] = synth.activation_bf16(synth.config_seed(CFG_INDEX, 1) + off, TOKENS, 2048)
+    host["x_down"] = synth.activation_bf16(synth.config_seed(CFG_INDEX, 7) + off, TOKENS, 11008)
+
+    def pinned(a):
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.pin_memory()
+
+    return {k: pinned(v) for k, v in host.items()}
+
+
+class Step:
+    """Device buffers and the launches of one training step of the three linears."""
+
+    def __init__(self, host, dev, n_keep=N_KEEP, m_group=M_GROUP):
+        import torch
+
+        import sparsity_step_b200 as B
+
+        self.B = B
+        self.n_keep, self.m_group = n_keep, m_group
+        bf = torch.bfloat16
+        self.d = {}
+        for k, v in host.items():
+            t = v.to(dev, non_blocking=False)
+            self.d[k] = t.view(bf) if v.dtype == torch.int16 else t
+        T = TOKENS
+        self.qm = {}
+        self.ws_qm = {}
+        for name, k_in, n_out in LINEARS:
+            self.qm[name] = {
+                "codes": torch.empty((n_out, k_in // 4), dtype=torch.uint8, device=dev),
+                "mask": torch.empty((n_out, k_in // m_group), dtype=torch.uint8, device=dev),
+                "w_i8": torch.empty((n_out, k_in), dtype=torch.int8, device=dev),
+                "w_scale": torch.empty((4,), dtype=torch.float32, device=dev)[:1],
+            }
+            self.ws_qm[name] = torch.empty((B.bitlinear_quant_mask_workspace_size(n_out, k_in),), dtype=torch.uint8,
+                                           device=dev)
+        self.xq_in = torch.empty((T, 2048), dtype=torch.int8, device=dev)
+        self.a_in = torch.empty((T,), dtype=torch.float32, device=dev)
+        self.xq_down = torch.empty((T, 11008), dtype=torch.int8, device=dev)
+        self.a_down = torch.empty((T,), dtype=torch.float32, device=dev)
+        self.y = {n: torch.empty((T, n_out), dtype=bf, device=dev) for n, _, n_out in LINEARS}
+        self.gx = {n: torch.empty((T, k_in), dtype=bf, device=dev) for n, k_in, _ in LINEARS}
+        self.gw = {n: torch.empty((n_out, k_in), dtype=bf, device=dev) for n, k_in, n_out in LINEARS}
+        wsb = max(B.bitlinear_bwd_workspace_size(T, k, n, True) for _, k, n in LINEARS)
+        self.ws_bwd = torch.empty((wsb,), dtype=torch.uint8, device=dev)
+        self.launches_per_step = 3 * 3 + 2 + 3 + 3 * 3
+
+    def run(self, ev=None):
+        """Enqueue one step. ``ev`` maps a kernel class to a list that receives
+        (start, end) CUDA events around each of its launches."""
+        import torch
+
+        B = self.B
+
+        def timed(key, fn):
+            if ev is None:
+                fn()
+                return
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            ev.setdefault(key, []).append((s, e))
+
+        for name, _, _ in LINEARS:
+            q = self.qm[name]
+            timed("quant_mask", lambda: B.bitlinear_quant_mask(self.d[f"w_{name}"], self.n_keep, self.m_group, out=q,
+                                                               workspace=self.ws_qm[name]))
+        timed("act_quant", lambda: B.bitlinear_act_quant(self.d["x_in"], xq=self.xq_in, absmax=self.a_in))
+        timed("act_quant", lambda: B.bitlinear_act_quant(self.d["x_down"], xq=self.xq_down, absmax=self.a_down))
+        for name, _, _ in LINEARS:
+            xq, a = (self.xq_down, self.a_down) if name == "down" else (self.xq_in, self.a_in)
+            q = self.qm[name]
+            timed("fwd_i8_gemm", lambda: B.bitlinear_fwd(xq, a, q["w_scale"], w_i8=q["w_i8"], y=self.y[name]))
+        for name, k_in, _ in LINEARS:
+            x = self.d["x_down"] if name == "down" else self.d["x_in"]
+            q = self.qm[name]
+            dy = self.d[f"dy_{name}"]
+            timed("bwd_grad_x", lambda: B.bitlinear_bwd(dy, None, q["codes"], q["w_scale"], want_grad_w=False,
+                                                        grad_x=self.gx[name], workspace=self.ws_bwd, k_in=k_in))
+            timed("bwd_grad_w", lambda: B.bitlinear_bwd(dy, x, None, None, want_grad_x=False, grad_w=self.gw[name]))
+
+    # bytes moved per step by the end-to-end variant
+    def e2e_inputs(self):
+        return ["x_in", "x_down"] + [f"dy_{n}" for n, _, _ in LINEARS]
+
+    def e2e_outputs(self):
+        return [self.y[n] for n, _, _ in LINEARS] + [self.gx[n] for n, _, _ in LINEARS]
+
+
+def algorithmic_counts():
+    """Per-step operation counts (dense-equivalent) of the step's products."""
+    fwd_ops = sum(2 * TOKENS * k * n for _, k, n in LINEARS)
+    bwd_flops = 2 * fwd_ops
+    return fwd_ops, bwd_flops
+
+
+def run_ours(args) -> None:
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    host = make_inputs(rank)
+    step = Step(host, dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+
+    # ---------------- device-resident timed region (kernel events inside)
+    ev = {}
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_smi_id(local)) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step.run(ev)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    ms_step = ms_total / args.steps
+    per_kernel_ms = {k: sum(s.elapsed_time(e) for s, e in v) / args.steps for k, v in ev.items()}
+    per_launch_ms = {k: sum(s.elapsed_time(e) for s, e in v) / len(v) for k, v in ev.items()}
+    clocks = clk.summary()
+
+    # status of the device-side checks (timeouts, weight range)
+    st, bits = step.B.bitlinear_device_status()
+    for name, _, _ in LINEARS:
+        if step.B.bitlinear_quant_mask_status(step.ws_qm[name]) != 0:
+            raise RuntimeError(f"weight range error in {name}")
+    if st != 0:
+        raise RuntimeError(f"device status {bits:#x}")
+
+    # ---------------- 6:8 versus 8:8 (same step, no mask)
+    dense = Step(host, dev, n_keep=8, m_group=8)
+    for _ in range(args.warmup):
+        dense.run()
+    barrier()
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(args.steps):
+        dense.run()
+    d1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_dense = max_over_ranks(d0.elapsed_time(d1)) / args.steps
+    del dense
+
+    # ---------------- end to end: pinned host inputs -> device -> step -> host outputs
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in step.e2e_outputs()]
+    h2d = sum(host[k].numel() * host[k].element_size() for k in step.e2e_inputs())
+    d2h = sum(t.numel() * t.element_size() for t in outs_host)
+
+    def e2e_step():
+        for k in step.e2e_inputs():
+            step.d[k].view(torch.int16).copy_(host[k], non_blocking=True)
+        step.run()
+        for hdst, dsrc in zip(outs_host, step.e2e_outputs()):
+            hdst.copy_(dsrc, non_blocking=True)
+
+    for _ in range(min(args.warmup, 3)):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+
+    # ---------------- roofline of the dominant kernel
+    peaks = load_peaks()
+    fwd_ops, bwd_flops = algorithmic_counts()
+    dominant = max(per_kernel_ms, key=per_kernel_ms.get)
+    gemm_flops_per_launch = 2 * TOKENS * 2048 * 11008          # every product here has this size
+    roof = None
+    if dominant in ("bwd_grad_w", "bwd_grad_x"):
+        achieved = gemm_flops_per_launch / (per_launch_ms[dominant] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        tr = TRAFFIC.get(dominant)
+        roof = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "peak_kind": f"bf16 sustained ({peaks['source']})",
+                "traffic": tr["bytes"] if tr and tr["sha"] == kernel_source_sha() else None,
+                "algorithmic_per_launch": gemm_flops_per_launch}
+    else:
+        roof = {"kernel": dominant, "bound": "unknown"}
+
+    tok_s = TOKENS * world / (ms_step * 1e-3)
+    out = {
+        "metric": METRIC,
+        "value": round(tok_s, 1),
+        "unit": "tok/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8+bf16",
+        "data": "synthetic (seeded N(0,0.02) fp32 latent W; N(0,1) bf16 X with 1% x20 outliers; N(0,1e-2) bf16 dY)",
+        "config": {"workload": WORKLOAD, "tokens_per_gpu": TOKENS, "nm": f"{N_KEEP}:{M_GROUP}",
+                   "linears": [f"{n} {k}->{o}" for n, k, o in LINEARS], "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (per-step working set ~1.5 GB vs 126 MB L2); no flush"},
+        "tops": {"fwd_int8_dense_equiv": round(fwd_ops / (per_kernel_ms["fwd_i8_gemm"] * 1e-3) / 1e12, 1),
+                 "fwd_int8_useful_6of8": round(fwd_ops * N_KEEP / M_GROUP / (per_kernel_ms["fwd_i8_gemm"] * 1e-3) / 1e12, 1),
+                 "bwd_bf16": round(bwd_flops / ((per_kernel_ms["bwd_grad_x"] + per_kernel_ms["bwd_grad_w"]) * 1e-3) / 1e12, 1),
+                 "int8_peak_from_bf16_x2": round(2 * peaks["bf16_tflops_sustained"], 1)},
+        "breakdown_ms_per_step": {k: round(v, 4) for k, v in per_kernel_ms.items()},
+        "speedup_vs_8_8": round(ms_dense / ms_step, 4),
+        "ms_per_step_8_8": round(ms_dense, 4),
+        "roofline": roof,
+        "e2e": {"value": round(TOKENS * world / (ms_e2e * 1e-3), 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 3), "steps": e2e_steps},
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.cpu_tokens)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arm
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(tokens: int, w_rows: int | None, seed_off: int = 0) -> dict:
+    """Time the oracle on a bounded sample: the mask/code recompute of the three
+    weight tensors (all rows, or the first ``w_rows``), and ``tokens`` tokens through
+    act-quant, forward and both gradients. Returns the seconds of each part."""
+    from oracle import bitlinear_oracle as O
+    from sparsity_step_b200 import synth
+
+    t_mask = 0.0
+    t_tok = 0.0
+    for i, (name, k_in, n_out) in enumerate(LINEARS):
+        rows = n_out if w_rows is None else min(w_rows, n_out)
+        w = synth.latent_weight(synth.config_seed(CFG_INDEX, 3 * i) + seed_off, rows, k_in)
+        x = synth.activation_bf16(synth.config_seed(CFG_INDEX, 3 * i + 1) + seed_off, tokens, k_in)
+        dy = synth.activation_bf16(synth.config_seed(CFG_INDEX, 3 * i + 2) + seed_off, tokens, n_out, std=1e-2,
+                                   outliers=False)
+        s = time.perf_counter()
+        qm = O.quant_mask(w, N_KEEP, M_GROUP)
+        t_mask += (time.perf_counter() - s) * (n_out / rows)
+        # the token part runs against a full-size code matrix
+        mcode = qm["mcode"] if rows == n_out else _tile_rows(qm["mcode"], n_out)
+        s = time.perf_counter()
+        q, a = O.act_quant(x)
+        O.fwd(q, a, mcode, qm["gamma"])
+        O.grad_x(dy, mcode, qm["gamma"])
+        O.grad_w(dy, x)
+        t_tok += time.perf_counter() - s
+    step_s = t_mask + t_tok * (TOKENS / tokens)
+    return {"mask_s": t_mask, "tokens_s": t_tok, "step_s": step_s}
+
+
+def _tile_rows(a, n):
+    import numpy as np
+    reps = (n + a.shape[0] - 1) // a.shape[0]
+    return np.ascontiguousarray(np.tile(a, (reps, 1))[:n])
+
+
+def cpu_baseline(tokens: int) -> dict:
+    r = oracle_sample(tokens, None)
+    return {"value": round(TOKENS / r["step_s"], 2), "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": (f"full mask/ternary recompute of the 3 weight tensors ({r['mask_s']:.2f} s) + {tokens} of "
+                       f"{TOKENS} tokens through act-quant/fwd/grad_x/grad_w ({r['tokens_s']:.2f} s), "
+                       f"step time extrapolated linearly in tokens")}
+
+
+def run_reference(args) -> None:
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    tokens, w_rows = args.ref_tokens, args.ref_w_rows
+    for _ in range(args.warmup):
+        oracle_sample(tokens, w_rows)
+    step_s = []
+    for _ in range(args.steps):
+        step_s.append(oracle_sample(tokens, w_rows)["step_s"])
+    ms = 1e3 * statistics.mean(step_s)
+    v = round(TOKENS / (ms * 1e-3), 3)
+    out = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64+f32 (oracle)", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_gpu": TOKENS, "nm": f"{N_KEEP}:{M_GROUP}",
+                   "linears": [f"{n} {k}->{o}" for n, k, o in LINEARS], "parallelism": "single process (CPU)"},
+        "cpu_baseline": {"value": v, "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": (f"each step: mask/ternary recompute of the first {w_rows} rows of each weight "
+                                    f"tensor (scaled to all rows) + {tokens} tokens through act-quant/fwd/grad_x/"
+                                    f"grad_w (scaled to {TOKENS} tokens)")},
+        "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-tokens", type=int, default=256, help="tokens in the oracle's timed sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=16, help="reference arm: tokens per sampled step")
+    ap.add_argument("--ref-w-rows", type=int, default=256, help="reference arm: weight rows per sampled step")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

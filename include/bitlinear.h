@@ -26,7 +26,8 @@
  *     stream). Calls only enqueue work and return; results are ready when the
  *     stream reaches them.
  *   - Shapes: k_in % 64 == 0, 64 <= k_in <= 131072, n_out % 16 == 0, n_out >= 16,
- *     t >= 0 (t = 0 is a valid empty batch). Else BL_ERR_UNSUPPORTED_SHAPE.
+ *     t >= 0 (t = 0 is a valid empty batch; the arrays sized by t may then be
+ *     NULL). Else BL_ERR_UNSUPPORTED_SHAPE.
  *   - bf16 arrays are passed as uint16_t bit patterns.
  *   - Errors: argument, shape and alignment errors return before anything is
  *     enqueued; a failed launch returns BL_ERR_CUDA. bitlinear_last_error() gives a

@@ -187,11 +187,11 @@ bl_status bitlinear_quant_mask_status(const void* workspace, void* stream) {
 
 bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t* xq_out, float* absmax_out, void* stream) {
   g_err[0] = 0;
-  if (!x || !xq_out || !absmax_out) return fail(BL_ERR_INVALID_ARG, "x, xq_out, absmax_out are required");
   if (bl_status s = check_shape(t, k_in, 16)) return s;
+  if (t == 0) return BL_OK;   // empty batch: the t-sized arrays may be NULL
+  if (!x || !xq_out || !absmax_out) return fail(BL_ERR_INVALID_ARG, "x, xq_out, absmax_out are required");
   if (!aligned16(x) || !aligned16(xq_out) || !aligned16(absmax_out))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
-  if (t == 0) return BL_OK;
   cudaStream_t st = as_stream(stream);
   const int k8 = static_cast<int>(k_in / 8);
   const uint4* xv = reinterpret_cast<const uint4*>(x);
@@ -217,14 +217,16 @@ bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* co
                         const float* w_scale, int64_t t, int64_t k_in, int64_t n_out, int32_t* acc_out, void* y_out,
                         int y_dtype, void* stream) {
   g_err[0] = 0;
-  if (!xq || !absmax || !w_scale || !y_out) return fail(BL_ERR_INVALID_ARG, "xq, absmax, w_scale, y_out are required");
+  if (!w_scale) return fail(BL_ERR_INVALID_ARG, "w_scale is required");
   if (!codes && !w_i8) return fail(BL_ERR_INVALID_ARG, "give codes or w_i8");
   if (y_dtype != BL_OUT_BF16 && y_dtype != BL_OUT_F32) return fail(BL_ERR_INVALID_ARG, "y_dtype must be BL_OUT_BF16 or BL_OUT_F32");
   if (bl_status s = check_shape(t, k_in, n_out)) return s;
-  if (!aligned16(xq) || !aligned16(absmax) || !aligned16(w_scale) || !aligned16(y_out) || (codes && !aligned16(codes)) ||
-      (w_i8 && !aligned16(w_i8)) || (acc_out && !aligned16(acc_out)))
+  if (!aligned16(w_scale) || (codes && !aligned16(codes)) || (w_i8 && !aligned16(w_i8)))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
-  if (t == 0) return BL_OK;
+  if (t == 0) return BL_OK;   // empty batch: the t-sized arrays may be NULL
+  if (!xq || !absmax || !y_out) return fail(BL_ERR_INVALID_ARG, "xq, absmax, y_out are required");
+  if (!aligned16(xq) || !aligned16(absmax) || !aligned16(y_out) || (acc_out && !aligned16(acc_out)))
+    return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
   cudaStream_t st = as_stream(stream);
   if (w_i8) {
     CUtensorMap ta, tb;
@@ -263,13 +265,13 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* co
                         size_t workspace_bytes, void* stream) {
   g_err[0] = 0;
   if (!grad_x && !grad_w) return fail(BL_ERR_INVALID_ARG, "request grad_x, grad_w or both");
-  if (!dy) return fail(BL_ERR_INVALID_ARG, "dy is required");
+  if (!dy && t != 0) return fail(BL_ERR_INVALID_ARG, "dy is required");
   if (grad_x && (!codes || !w_scale)) return fail(BL_ERR_INVALID_ARG, "grad_x needs codes and w_scale");
-  if (grad_w && !x) return fail(BL_ERR_INVALID_ARG, "grad_w needs x");
+  if (grad_w && !x && t != 0) return fail(BL_ERR_INVALID_ARG, "grad_w needs x");
   if (grad_w && grad_w_dtype != BL_OUT_BF16 && grad_w_dtype != BL_OUT_F32)
     return fail(BL_ERR_INVALID_ARG, "grad_w_dtype must be BL_OUT_BF16 or BL_OUT_F32");
   if (bl_status s = check_shape(t, k_in, n_out)) return s;
-  if (!aligned16(dy) || (x && !aligned16(x)) || (codes && !aligned16(codes)) || (w_scale && !aligned16(w_scale)) ||
+  if ((dy && !aligned16(dy)) || (x && !aligned16(x)) || (codes && !aligned16(codes)) || (w_scale && !aligned16(w_scale)) ||
       (grad_x && !aligned16(grad_x)) || (grad_w && !aligned16(grad_w)) || (workspace && !aligned16(workspace)))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
   const size_t need = bitlinear_bwd_workspace_size(t, k_in, n_out, grad_x != nullptr);
