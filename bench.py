@@ -480,6 +480,58 @@ def run_reference(args) -> None:
     print(json.dumps(out), flush=True)
 
 
+def run_case(args) -> None:
+    """One kernel class alone on a chosen shape (for ncu captures and tuning):
+    warm-up launches, then ``--steps`` timed launches; prints one JSON line."""
+    import numpy as np
+    import torch
+
+    import sparsity_step_b200 as B
+    from sparsity_step_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    t, k_in, n_out = args.case_t, args.case_k, args.case_n
+    w = torch.from_numpy(synth.latent_weight(11, n_out, k_in)).to(dev)
+
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    x = bf(synth.activation_bf16(12, t, k_in))
+    dy = bf(synth.activation_bf16(13, t, n_out, std=1e-2, outliers=False))
+    qm = B.bitlinear_quant_mask(w, N_KEEP, M_GROUP)
+    xq, a = B.bitlinear_act_quant(x)
+    y = torch.empty((t, n_out), dtype=torch.bfloat16, device=dev)
+    gx = torch.empty((t, k_in), dtype=torch.bfloat16, device=dev)
+    gw = torch.empty((n_out, k_in), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((B.bitlinear_bwd_workspace_size(t, k_in, n_out, True),), dtype=torch.uint8, device=dev)
+    flops = 2.0 * t * k_in * n_out
+    cases = {
+        "quant_mask": (lambda: B.bitlinear_quant_mask(w, N_KEEP, M_GROUP, out=qm, workspace=qm["workspace"]),
+                       "GB/s", n_out * k_in * (4 + 4 + 1 + 0.25 + 0.125)),
+        "act_quant": (lambda: B.bitlinear_act_quant(x, xq=xq, absmax=a), "GB/s", t * k_in * 3 + 4 * t),
+        "fwd": (lambda: B.bitlinear_fwd(xq, a, qm["w_scale"], w_i8=qm["w_i8"], y=y), "TOP/s", flops),
+        "fwd_codes": (lambda: B.bitlinear_fwd(xq, a, qm["w_scale"], codes=qm["codes"], y=y), "GB/s",
+                      n_out * k_in / 4 + t * k_in + 2 * t * n_out),
+        "grad_x": (lambda: B.bitlinear_bwd(dy, None, qm["codes"], qm["w_scale"], want_grad_w=False, grad_x=gx,
+                                           workspace=ws, k_in=k_in), "TFLOP/s", flops),
+        "grad_w": (lambda: B.bitlinear_bwd(dy, x, None, None, want_grad_x=False, grad_w=gw), "TFLOP/s", flops),
+    }
+    fn, unit, work = cases[args.case]
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / args.steps
+    rate = work / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+    print(json.dumps({"case": args.case, "t": t, "k_in": k_in, "n_out": n_out, "ms_per_launch": round(ms, 5),
+                      "rate": round(rate, 1), "unit": unit}), flush=True)
+
+
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -491,7 +543,15 @@ def main(argv=None) -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=16, help="reference arm: tokens per sampled step")
     ap.add_argument("--ref-w-rows", type=int, default=256, help="reference arm: weight rows per sampled step")
+    ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_codes", "grad_x", "grad_w"],
+                    help="time one kernel class alone on the --case-t/k/n shape")
+    ap.add_argument("--case-t", type=int, default=TOKENS)
+    ap.add_argument("--case-k", type=int, default=2048)
+    ap.add_argument("--case-n", type=int, default=11008)
     args = ap.parse_args(argv)
+    if args.case:
+        run_case(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
