@@ -96,6 +96,27 @@ bl_status bitlinear_quant_mask(const float* w_latent, int64_t n_out, int64_t k_i
 bl_status bitlinear_quant_mask_status(const void* workspace, void* stream);
 
 /*
+ * bitlinear_quant_mask without a workspace and without any allocation. The paper has
+ * no counterpart: this is a library convenience. It is for callers that cannot
+ * allocate device memory at all -- code running inside a host framework that owns
+ * every byte of device memory, or a latency-critical path where cudaMalloc/cudaFree
+ * (which may synchronise the device) are not allowed.
+ *
+ * Same computation, arguments and outputs as bitlinear_quant_mask, minus the
+ * workspace. Its scratch is a fixed array of 19200 bytes inside the library (every
+ * GPU that loads the library holds it until exit), which limits the tensor to
+ * n_out * k_in <= 4966055936 weights; larger tensors get BL_ERR_UNSUPPORTED_SHAPE.
+ * The first call on each device looks up that array's device address (with the
+ * device current); make that first call before any stream capture. All calls on a
+ * device share the array, so calls that overlap on the GPU race: order them on one
+ * stream. A range error shows as gamma = NaN and all-zero codes (there is no
+ * workspace to read a status from).
+ */
+bl_status bitlinear_quant_mask_noalloc(const float* w_latent, int64_t n_out, int64_t k_in, int n_keep, int m_group,
+                                       uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out, float* w_scale_out,
+                                       void* stream);
+
+/*
  * Step a3: per-token absmax int8 activation quantisation of X [t, k_in] (bf16).
  *   a_t = max_k |x_tk|   (a zero row uses a_t = 1e-5, giving q = 0)
  *   q   = clamp(rint(x * fp32(127 / a_t)), -128, 127), one fp32 multiply, ties to even.

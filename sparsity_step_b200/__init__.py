@@ -13,6 +13,7 @@ from .bitlinear import (  # noqa: F401
     bitlinear_device_status,
     bitlinear_fwd,
     bitlinear_quant_mask,
+    bitlinear_quant_mask_noalloc,
     bitlinear_quant_mask_status,
     bitlinear_quant_mask_workspace_size,
 )

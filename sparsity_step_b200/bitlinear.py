@@ -76,6 +76,23 @@ def bitlinear_quant_mask_status(workspace: torch.Tensor, stream=None) -> int:
     return int(lib().bitlinear_quant_mask_status(_ptr(workspace), _stream(stream)))
 
 
+def bitlinear_quant_mask_noalloc(w: torch.Tensor, n_keep: int, m_group: int, *, out: dict, stream=None) -> dict:
+    """bitlinear_quant_mask with no workspace and no allocation inside the library.
+
+    For callers that cannot allocate device memory: every output buffer comes in
+    ``out`` (``codes``, ``w_scale``, and optionally ``mask`` and ``w_i8``); the
+    library's built-in scratch array is used instead of a workspace. Calls that
+    overlap on the GPU share that array and race; a range error gives gamma = NaN.
+    """
+    n_out, k_in = w.shape
+    _need(w, torch.float32, None, "w")
+    st = lib().bitlinear_quant_mask_noalloc(_ptr(w), n_out, k_in, n_keep, m_group, _ptr(out.get("mask")),
+                                            _ptr(out["codes"]), _ptr(out.get("w_i8")), _ptr(out["w_scale"]),
+                                            _stream(stream))
+    check(st, "bitlinear_quant_mask_noalloc")
+    return out
+
+
 def bitlinear_act_quant(x: torch.Tensor, *, xq: torch.Tensor | None = None, absmax: torch.Tensor | None = None,
                         stream=None) -> tuple[torch.Tensor, torch.Tensor]:
     """int8 activations and per-token absmax of x [t, k_in] (bf16)."""
@@ -152,6 +169,7 @@ def bitlinear_abi_version() -> int:
 
 __all__ = [
     "bitlinear_quant_mask_workspace_size", "bitlinear_quant_mask", "bitlinear_quant_mask_status",
+    "bitlinear_quant_mask_noalloc",
     "bitlinear_act_quant", "bitlinear_fwd", "bitlinear_bwd_workspace_size", "bitlinear_bwd",
     "bitlinear_device_status", "bitlinear_abi_version", "BL_OUT_BF16", "BL_OUT_F32", "_lib",
 ]

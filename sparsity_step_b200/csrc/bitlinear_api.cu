@@ -344,3 +344,95 @@ bl_status bitlinear_device_status(unsigned int* bits) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ quant_mask without allocation
+//
+// Some callers cannot allocate device memory at all: code that runs inside a host
+// framework owning every byte of device memory (a fixed arena or a caching pool that
+// forbids outside cudaMalloc), and latency-critical paths where cudaMalloc/cudaFree
+// (which may synchronise the whole device) are not allowed. For them,
+// bitlinear_quant_mask_noalloc keeps its scratch (range flag, status word and the
+// per-block partial sums) in the file-scope array below instead of a caller workspace.
+//
+// The array is a host-side stand-in in host code: its device address is fetched with
+// cudaGetSymbolAddress once per device (with that device current) on the first call
+// made on that device, and that address is what the kernels receive. Every call on a
+// device shares the array: calls that overlap on the GPU (different streams, no
+// ordering between them) race on it. Each call clears the header it needs at zero.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 19200;   // 256-byte header + 16 B x 1184 block partials
+static __device__ __align__(256) unsigned char g_qm_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+bl_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(BL_ERR_INVALID_ARG, "device ordinal %d not supported", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_qm_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BL_OK;
+}
+
+}  // namespace
+
+extern "C" bl_status bitlinear_quant_mask_noalloc(const float* w_latent, int64_t n_out, int64_t k_in, int n_keep,
+                                                  int m_group, uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out,
+                                                  float* w_scale_out, void* stream) {
+  g_err[0] = 0;
+  if (!w_latent || !codes_out || !w_scale_out) return fail(BL_ERR_INVALID_ARG, "w_latent, codes_out, w_scale_out are required");
+  if (bl_status s = check_shape(0, k_in, n_out)) return s;
+  if (!(m_group == 4 || m_group == 8) || n_keep < 1 || n_keep > m_group)
+    return fail(BL_ERR_INVALID_ARG, "N:M = %d:%d: need M in {4, 8} and 1 <= N <= M", n_keep, m_group);
+  const int64_t numel = n_out * k_in;
+  const size_t need = bitlinear_quant_mask_workspace_size(n_out, k_in);
+  if (need > kNoAllocScratchBytes)
+    return fail(BL_ERR_UNSUPPORTED_SHAPE,
+                "tensor of %lld weights needs %zu scratch bytes; the built-in scratch holds %zu "
+                "(at most 4966055936 weights): use bitlinear_quant_mask with a workspace",
+                (long long)numel, need, kNoAllocScratchBytes);
+  if (!aligned16(w_latent) || !aligned16(codes_out) || !aligned16(w_scale_out) || (mask_out && !aligned16(mask_out)) ||
+      (w_i8_out && !aligned16(w_i8_out)))
+    return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  void* scratch = nullptr;
+  if (bl_status s = noalloc_scratch(&scratch)) return s;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  unsigned int* range_flag = reinterpret_cast<unsigned int*>(ws);
+  int* status = reinterpret_cast<int*>(ws + 4);
+  unsigned long long* partials = reinterpret_cast<unsigned long long*>(ws + bl::kQmWsHeader);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 16, st);   // range flag and status start at zero
+  if (e != cudaSuccess) return cuda_fail(e, "scratch reset");
+  const int blocks = qm_blocks(numel);
+  bl::qm_abs_sum_kernel<<<blocks, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), numel / 4, partials,
+                                                          range_flag);
+  bl::qm_finalize_kernel<<<1, 256, 0, st>>>(partials, blocks, numel, range_flag, status, w_scale_out);
+  const int64_t n8 = numel / 8;
+  int64_t g2 = (n8 + bl::kQmThreads - 1) / bl::kQmThreads;
+  const int64_t cap = int64_t(device_sm_count()) * 16;
+  if (g2 > cap) g2 = cap;
+  if (m_group == 8)
+    bl::qm_mask_codes_kernel<8><<<(int)g2, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), n8, n_keep,
+                                                                     w_scale_out, mask_out,
+                                                                     reinterpret_cast<uint16_t*>(codes_out),
+                                                                     reinterpret_cast<uint2*>(w_i8_out));
+  else
+    bl::qm_mask_codes_kernel<4><<<(int)g2, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), n8, n_keep,
+                                                                     w_scale_out, mask_out,
+                                                                     reinterpret_cast<uint16_t*>(codes_out),
+                                                                     reinterpret_cast<uint2*>(w_i8_out));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quant_mask_noalloc launch");
+  return BL_OK;
+}

@@ -53,6 +53,16 @@ def test_quant_mask_validation(L):
     assert "aligned" in _err(L)
 
 
+def test_quant_mask_noalloc_validation(L):
+    assert L.bitlinear_quant_mask_noalloc(None, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, None) == -1
+    assert L.bitlinear_quant_mask_noalloc(GOOD, 896, 896, 9, 8, GOOD, GOOD, GOOD, GOOD, None) == -1
+    assert L.bitlinear_quant_mask_noalloc(GOOD, 896, 900, 6, 8, GOOD, GOOD, GOOD, GOOD, None) == -2
+    # beyond the built-in scratch (1184 block partials): rejected on the host
+    assert L.bitlinear_quant_mask_noalloc(GOOD, 1 << 20, 8192, 6, 8, None, GOOD, None, GOOD, None) == -2
+    assert "scratch" in _err(L)
+    assert L.bitlinear_quant_mask_noalloc(BAD, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, None) == -3
+
+
 def test_act_quant_validation(L):
     assert L.bitlinear_act_quant(None, 4, 896, GOOD, GOOD, None) == -1
     assert L.bitlinear_act_quant(GOOD, 4, 100, GOOD, GOOD, None) == -2
