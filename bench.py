@@ -342,6 +342,12 @@ def run_ours(args) -> None:
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
 
+    # ---------------- raw tensor-pipe rates of this GPU (probe: MMAs from shared memory only)
+    try:
+        probe = {"int8_tops": round(mma_peak("i8"), 1), "bf16_tflops": round(mma_peak("bf16"), 1)}
+    except (OSError, RuntimeError) as exc:
+        probe = {"error": str(exc)}
+
     # ---------------- roofline of the dominant kernel
     peaks = load_peaks()
     fwd_ops, bwd_flops = algorithmic_counts()
@@ -379,7 +385,8 @@ def run_ours(args) -> None:
         "tops": {"fwd_int8_dense_equiv": round(fwd_ops / (per_kernel_ms["fwd_i8_gemm"] * 1e-3) / 1e12, 1),
                  "fwd_int8_useful_6of8": round(fwd_ops * N_KEEP / M_GROUP / (per_kernel_ms["fwd_i8_gemm"] * 1e-3) / 1e12, 1),
                  "bwd_bf16": round(bwd_flops / ((per_kernel_ms["bwd_grad_x"] + per_kernel_ms["bwd_grad_w"]) * 1e-3) / 1e12, 1),
-                 "int8_peak_from_bf16_x2": round(2 * peaks["bf16_tflops_sustained"], 1)},
+                 "int8_peak_from_bf16_x2": round(2 * peaks["bf16_tflops_sustained"], 1),
+                 "tensor_pipe_probe": probe},
         "breakdown_ms_per_step": {k: round(v, 4) for k, v in per_kernel_ms.items()},
         "speedup_vs_8_8": round(ms_dense / ms_step, 4),
         "ms_per_step_8_8": round(ms_dense, 4),
@@ -480,6 +487,36 @@ def run_reference(args) -> None:
     print(json.dumps(out), flush=True)
 
 
+def mma_peak(kind: str, iters: int = 4000, reps: int = 3) -> float:
+    """Dense tcgen05 MMA rate (TOP/s or TFLOP/s) of this GPU from the probe library:
+    148 CTAs issuing back-to-back 128x256 MMAs from shared memory (no memory traffic)."""
+    import ctypes
+
+    import torch
+
+    lib = ctypes.CDLL(os.path.join(ROOT, "sparsity_step_b200", "libblprobe.so"))
+    lib.blprobe_mma_peak.restype = ctypes.c_int
+    lib.blprobe_mma_peak.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    k = 1 if kind == "i8" else 0
+    ctas = torch.cuda.get_device_properties(0).multi_processor_count
+    st = torch.cuda.current_stream()
+    if lib.blprobe_mma_peak(k, ctas, 100, st.cuda_stream) != 0:
+        raise RuntimeError("mma probe failed")
+    best = 0.0
+    for _ in range(reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(st)
+        rc = lib.blprobe_mma_peak(k, ctas, iters, st.cuda_stream)
+        e.record(st)
+        torch.cuda.synchronize()
+        if rc != 0:
+            raise RuntimeError(f"mma probe failed ({rc})")
+        kdim = 32 if kind == "i8" else 16
+        ops = 2.0 * 128 * 256 * kdim * 4 * iters * ctas
+        best = max(best, ops / (s.elapsed_time(e) * 1e-3) / 1e12)
+    return best
+
+
 def run_case(args) -> None:
     """One kernel class alone on a chosen shape (for ncu captures and tuning):
     warm-up launches, then ``--steps`` timed launches; prints one JSON line."""
@@ -489,6 +526,11 @@ def run_case(args) -> None:
     import sparsity_step_b200 as B
     from sparsity_step_b200 import synth
 
+    if args.case.startswith("mma_peak"):
+        kind = args.case.split("_")[-1]
+        print(json.dumps({"case": args.case, "rate": round(mma_peak(kind), 1),
+                          "unit": "TOP/s" if kind == "i8" else "TFLOP/s"}), flush=True)
+        return
     dev = torch.device("cuda", 0)
     t, k_in, n_out = args.case_t, args.case_k, args.case_n
     w = torch.from_numpy(synth.latent_weight(11, n_out, k_in)).to(dev)
@@ -543,7 +585,8 @@ def main(argv=None) -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=16, help="reference arm: tokens per sampled step")
     ap.add_argument("--ref-w-rows", type=int, default=256, help="reference arm: weight rows per sampled step")
-    ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_codes", "grad_x", "grad_w"],
+    ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_codes", "grad_x", "grad_w", "mma_peak_i8",
+                             "mma_peak_bf16"],
                     help="time one kernel class alone on the --case-t/k/n shape")
     ap.add_argument("--case-t", type=int, default=TOKENS)
     ap.add_argument("--case-k", type=int, default=2048)

@@ -16,6 +16,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbitlinear.so")
 MAIN = os.path.join(CSRC, "bitlinear_api.cu")
+# measurement-only tensor-pipe probe (not part of the BitLinear ABI)
+PROBE_LIB = os.path.join(PKG, "libblprobe.so")
+PROBE_SRC = os.path.join(CSRC, "probe_mma_peak.cu")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -37,17 +40,15 @@ def sources() -> list[str]:
         os.path.join(ROOT, "include", "bitlinear.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = [nvcc_path(), *NVCC_FLAGS, *(extra or []), "-o", LIB + ".tmp", MAIN]
+def _nvcc(out: str, src: str, verbose: bool, extra: list[str] | None) -> None:
+    cmd = [nvcc_path(), *NVCC_FLAGS, *(extra or []), "-o", out + ".tmp", src]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -55,7 +56,14 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose and (res.stdout or res.stderr):
         print(res.stdout, res.stderr, sep="\n")
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(out + ".tmp", out)
+
+
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
+    if force or not up_to_date(LIB):
+        _nvcc(LIB, MAIN, verbose, extra)
+    if force or not up_to_date(PROBE_LIB):
+        _nvcc(PROBE_LIB, PROBE_SRC, verbose, extra)
     return LIB
 
 

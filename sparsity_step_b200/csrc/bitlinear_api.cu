@@ -82,18 +82,27 @@ bl_status make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const vo
   return BL_OK;
 }
 
-template <bool kI8, bool kAMN, bool kBMN, int kEpi>
-bl_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const bl::GemmArgs& g, cudaStream_t st) {
-  auto kern = bl::gemm_tc_kernel<kI8, kAMN, kBMN, kEpi>;
+// Output tensor map of the TMA-store epilogue: [M, N] row-major, boxes of 32 rows x
+// 128 bytes (64 bf16 or 32 fp32 columns), 128-byte swizzle.
+bl_status make_out_map(CUtensorMap* m, const void* out, int64_t rows, int64_t cols, bool f32) {
+  return make_map(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 4 : 2, out, cols, rows,
+                  f32 ? 32 : 64, 32);
+}
+
+template <bool kI8, bool kAMN, bool kBMN, int kEpi, bool kTmaStore>
+bl_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout, const bl::GemmArgs& g,
+                      cudaStream_t st) {
+  auto kern = bl::gemm_tc_kernel<kI8, kAMN, kBMN, kEpi, kTmaStore>;
+  constexpr size_t smem = bl::gemm_smem_bytes(kTmaStore);
   static bool attr_set = false;   // per instantiation; cheap to repeat if raced
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bl::kGemmSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
     attr_set = true;
   }
   const int tiles = g.num_m_blocks * g.num_n_blocks;
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  kern<<<grid, bl::kGemmThreads, bl::kGemmSmemBytes, st>>>(ta, tb, g);
+  kern<<<grid, bl::kGemmThreads, smem, st>>>(ta, tb, tout, g);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return BL_OK;
@@ -243,7 +252,12 @@ bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* co
     g.acc_out = acc_out;
     g.row_absmax = absmax;
     g.w_scale = w_scale;
-    return launch_gemm<true, false, false, bl::EPI_FWD>(ta, tb, g, st);
+    if (acc_out) {   // int32 accumulators requested: per-row direct stores of y and acc
+      return launch_gemm<true, false, false, bl::EPI_FWD, false>(ta, tb, ta, g, st);
+    }
+    CUtensorMap to;
+    if (bl_status s = make_out_map(&to, y_out, t, n_out, g.out_f32)) return s;
+    return launch_gemm<true, false, false, bl::EPI_FWD, true>(ta, tb, to, g, st);
   }
   const unsigned grid = static_cast<unsigned>((n_out + bl::kCodesWarps - 1) / bl::kCodesWarps);
   bl::fwd_codes_kernel<<<grid, bl::kCodesWarps * 32, 0, st>>>(xq, absmax, codes, w_scale, static_cast<int>(t),
@@ -309,7 +323,9 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* co
     g.out = grad_x;
     g.out_f32 = 0;
     g.w_scale = w_scale;
-    if (bl_status s = launch_gemm<false, false, true, bl::EPI_GRADX>(ta, tb, g, st)) return s;
+    CUtensorMap to;
+    if (bl_status s = make_out_map(&to, grad_x, t, k_in, false)) return s;
+    if (bl_status s = launch_gemm<false, false, true, bl::EPI_GRADX, true>(ta, tb, to, g, st)) return s;
   }
   if (grad_w) {
     CUtensorMap ta, tb;
@@ -324,7 +340,9 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* co
     g.num_n_blocks = static_cast<int>((k_in + bl::kBN - 1) / bl::kBN);
     g.out = grad_w;
     g.out_f32 = grad_w_dtype == BL_OUT_F32;
-    if (bl_status s = launch_gemm<false, true, true, bl::EPI_GRADW>(ta, tb, g, st)) return s;
+    CUtensorMap to;
+    if (bl_status s = make_out_map(&to, grad_w, n_out, k_in, g.out_f32)) return s;
+    if (bl_status s = launch_gemm<false, true, true, bl::EPI_GRADW, true>(ta, tb, to, g, st)) return s;
   }
   return BL_OK;
 }

@@ -37,7 +37,12 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kGemmThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBarrierBytes = 256;
-constexpr size_t kGemmSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kBarrierBytes;
+// epilogue staging for TMA stores: per epilogue warp two buffers of 32 rows x 128 B
+constexpr int kStageOutBytes = 32 * 128;
+constexpr int kOutStagingBytes = 4 * 2 * kStageOutBytes;   // 32 KB
+constexpr size_t gemm_smem_bytes(bool tma_store) {
+  return 1024 + static_cast<size_t>(kStages) * kStageBytes + (tma_store ? kOutStagingBytes : 0) + kBarrierBytes;
+}
 
 enum Epi : int { EPI_FWD = 0, EPI_GRADX = 1, EPI_GRADW = 2 };
 
@@ -103,9 +108,74 @@ __device__ __forceinline__ void epilogue_store32(const GemmArgs& g, const uint32
   }
 }
 
-template <bool kI8, bool kAMN, bool kBMN, int kEpi>
+// Epilogue of one tile row-quarter through shared memory and TMA stores: the warp
+// converts 32 rows x 128 B (64 bf16 or 32 fp32 columns) at a time into a 128B-swizzled
+// staging buffer (row r at r*128, 16-byte chunk j at position j ^ (r & 7): conflict-free
+// and the layout the store's tensor map expects), then one lane stores the box.
+template <int kEpi>
+__device__ __forceinline__ void epilogue_tile_tma(const GemmArgs& g, const CUtensorMap* tmOut, uint32_t t_row,
+                                                  uint32_t stage_base, int& cnt, int row0, int n0, float rs, int lane) {
+  const int ecols = g.out_f32 ? 32 : 64;
+  for (int c = 0; c < kBN / ecols; ++c, ++cnt) {
+    const uint32_t buf = stage_base + static_cast<uint32_t>(cnt & 1) * kStageOutBytes;
+    if (cnt >= 2) {
+      if (lane == 0) bulk_wait_group_read<1>();   // the store that last read this buffer is done reading
+      __syncwarp();
+    }
+    uint32_t r0[32], r1[32];
+    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * ecols), r0);
+    if (!g.out_f32) tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * ecols + 32), r1);
+    tmem_ld_wait();
+    uint32_t w[32];   // the 128 bytes of this thread's row
+    if (g.out_f32) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float f;
+        if (kEpi == EPI_FWD) f = __fmul_rn(static_cast<float>(static_cast<int32_t>(r0[j])), rs);
+        else if (kEpi == EPI_GRADX) f = __fmul_rn(__uint_as_float(r0[j]), rs);
+        else f = __uint_as_float(r0[j]);
+        w[j] = __float_as_uint(f);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const uint32_t a = j < 16 ? r0[2 * j] : r1[2 * j - 32];
+        const uint32_t b = j < 16 ? r0[2 * j + 1] : r1[2 * j - 31];
+        float fa, fb;
+        if (kEpi == EPI_FWD) {
+          fa = __fmul_rn(static_cast<float>(static_cast<int32_t>(a)), rs);
+          fb = __fmul_rn(static_cast<float>(static_cast<int32_t>(b)), rs);
+        } else if (kEpi == EPI_GRADX) {
+          fa = __fmul_rn(__uint_as_float(a), rs);
+          fb = __fmul_rn(__uint_as_float(b), rs);
+        } else {
+          fa = __uint_as_float(a);
+          fb = __uint_as_float(b);
+        }
+        w[j] = pack_bf16x2(fa, fb);
+      }
+    }
+    const uint32_t row_addr = buf + static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t dst = row_addr + static_cast<uint32_t>((j ^ (lane & 7)) * 16);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w[4 * j]), "r"(w[4 * j + 1]),
+                   "r"(w[4 * j + 2]), "r"(w[4 * j + 3])
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmOut, buf, n0 + c * ecols, row0);
+      bulk_commit_group();
+    }
+  }
+}
+
+template <bool kI8, bool kAMN, bool kBMN, int kEpi, bool kTmaStore>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmOut, const GemmArgs g) {
   static_assert(!(kI8 && (kAMN || kBMN)), "the int8 product uses K-major operands only");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -113,7 +183,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t sA = base;
   const uint32_t sB = base + kStages * kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  const uint32_t sOut = base + kStages * kStageBytes;   // epilogue staging (kTmaStore only)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + (kTmaStore ? kOutStagingBytes : 0));
   const uint32_t bar0 = smem_u32(bars);
   // barrier slots: full[kStages] | empty[kStages] | tmem_full[2] | tmem_empty[2] | done
   const uint32_t full0 = bar0, empty0 = bar0 + 8u * kStages;
@@ -136,6 +207,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (kTmaStore) tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -251,6 +323,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quad = warp & 3;   // TMEM lanes [32*quad, 32*quad+32) belong to this warp
     const int row_in_tile = quad * 32 + lane;
     const float gamma = (kEpi == EPI_GRADW) ? 1.0f : *g.w_scale;
+    const uint32_t stage_base = sOut + static_cast<uint32_t>((warp - 2) * 2 * kStageOutBytes);
+    int cnt = 0;   // staging buffers used so far (double-buffered)
     int local = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
@@ -273,13 +347,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         rs = gamma;
       }
       const uint32_t t_row = tmem_base + static_cast<uint32_t>(buf * kBN) + (static_cast<uint32_t>(quad * 32) << 16);
+      if (kTmaStore) {
+        epilogue_tile_tma<kEpi>(g, &tmOut, t_row, stage_base, cnt, row - lane, n0, rs, lane);
+      } else {
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), r);
-        tmem_ld_wait();
-        const int col0 = n0 + c * 32;
-        if (row_ok && col0 < g.N) epilogue_store32<kEpi>(g, r, row, col0, rs);
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), r);
+          tmem_ld_wait();
+          const int col0 = n0 + c * 32;
+          if (row_ok && col0 < g.N) epilogue_store32<kEpi>(g, r, row, col0, rs);
+        }
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -289,6 +367,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       *abort_flag = 1;
       atomicOr(&g_device_status, DEV_ST_TIMEOUT_EPILOGUE);
     }
+    if (kTmaStore && lane == 0) bulk_wait_group_all();   // stores complete before the CTA exits
   }
 
   __syncthreads();

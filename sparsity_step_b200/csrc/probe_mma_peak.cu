@@ -1,0 +1,90 @@
+// Tensor-pipe throughput probe (measurement only, not part of the BitLinear ABI):
+// every CTA issues back-to-back 128x256 tcgen05.mma instructions on operands that
+// stay in shared memory, so the result is the dense MMA rate of one B200 at the
+// clock it runs at, with no memory traffic. Built as libblprobe.so; bench.py uses it
+// to report the int8 and bf16 tensor peaks its roofline fractions refer to.
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int kProbeThreads = 128;
+constexpr int kProbeSmem = 1024 + 16384 + 32768 + 64;
+
+template <bool kI8>
+__global__ void __launch_bounds__(kProbeThreads, 1) mma_peak_kernel(int iters, unsigned int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = bl::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  // small finite operand values (int8 1, bf16 1.0 / 0) keep the accumulators finite
+  for (int i = threadIdx.x; i < (16384 + 32768) / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(smem)[i] = kI8 ? 0x01010101u : 0x00003F80u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 16384 + 32768);
+  const uint32_t bar = bl::smem_u32(tmem_slot + 2);
+  const int warp = threadIdx.x >> 5;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (threadIdx.x == 0) {
+    bl::mbar_init(bar, 1);
+    bl::fence_mbar_init();
+  }
+  if (warp == 0) {
+    bl::tmem_alloc(bl::smem_u32(tmem_slot), 512);
+    bl::tmem_relinquish();
+  }
+  bl::tc_fence_before_sync();
+  __syncthreads();
+  bl::tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) {
+    constexpr uint32_t idesc = kI8 ? bl::make_idesc(2u, 1u, 1u, 0u, 0u, 256, 128) : bl::make_idesc(1u, 1u, 1u, 0u, 0u, 256, 128);
+    for (int i = 0; i < iters; ++i) {
+      const uint32_t d = tmem + static_cast<uint32_t>((i & 1) * 256);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = bl::make_sw128_desc(base + kk * 32, 16, 1024);
+        const uint64_t bd = bl::make_sw128_desc(base + 16384 + kk * 32, 16, 1024);
+        if (kI8) bl::tc_mma_i8(d, ad, bd, idesc, (i > 1 || kk > 0) ? 1u : 0u);
+        else bl::tc_mma_f16(d, ad, bd, idesc, (i > 1 || kk > 0) ? 1u : 0u);
+      }
+    }
+    bl::tc_commit(bar);
+    const uint64_t t0 = bl::global_timer_ns();
+    while (!bl::mbar_try_wait(bar, 0)) {
+      if (bl::global_timer_ns() - t0 > bl::kWaitTimeoutNs) {
+        atomicOr(status, 1u);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    bl::tc_fence_after_sync();
+    bl::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+// Runs the probe: `kind` 0 = bf16 (kind::f16), 1 = int8 (kind::i8); `ctas` CTAs of
+// `iters` x 4 MMAs of 128x256x(16|32). Returns 0, or -1 on a CUDA error, -6 on a
+// timeout. The caller times it (CUDA events on `stream`).
+extern "C" int blprobe_mma_peak(int kind, int ctas, int iters, void* stream) {
+  static unsigned int* status = nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!status && cudaMalloc(&status, sizeof(unsigned int)) != cudaSuccess) return -1;
+  cudaMemsetAsync(status, 0, sizeof(unsigned int), st);
+  if (kind == 1) {
+    cudaFuncSetAttribute(mma_peak_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kProbeSmem);
+    mma_peak_kernel<true><<<ctas, kProbeThreads, kProbeSmem, st>>>(iters, status);
+  } else {
+    cudaFuncSetAttribute(mma_peak_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kProbeSmem);
+    mma_peak_kernel<false><<<ctas, kProbeThreads, kProbeSmem, st>>>(iters, status);
+  }
+  if (cudaGetLastError() != cudaSuccess) return -1;
+  unsigned int h = 0;
+  if (cudaMemcpyAsync(&h, status, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return -1;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return -1;
+  return h ? -6 : 0;
+}

@@ -55,6 +55,11 @@ def check_fwd(qm_dev, xq, a, ref_qm, ref_q, ref_a, tag, rows=None, paths=("w_i8"
             acc_np, ybits = acc_np[rows], ybits[rows]
         assert_exact(acc_np, acc_ref, f"{tag} acc [{path}]")
         assert_bf16_within_ulp(ybits, y_ref, f"{tag} y bf16 [{path}]")
+        # without the int32 output the tensor-core path stores y through TMA
+        y2, _ = B.bitlinear_fwd(xq, a, qm_dev["w_scale"], n_out=ref_qm["mcode"].shape[0], **kw)
+        torch.cuda.synchronize()
+        y2bits = bf16_dev_to_bits(y2)
+        assert_bf16_within_ulp(y2bits if rows is None else y2bits[rows], y_ref, f"{tag} y bf16 no-acc [{path}]")
         if f32:
             y32, _ = B.bitlinear_fwd(xq, a, qm_dev["w_scale"], n_out=ref_qm["mcode"].shape[0], y_dtype=torch.float32, **kw)
             torch.cuda.synchronize()
