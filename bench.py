@@ -155,9 +155,15 @@ def make_inputs(rank: int):
 
 
 class Step:
-    """Device buffers and the launches of one training step of the three linears."""
+    """Device buffers and the launches of one training step of the three linears.
 
-    def __init__(self, host, dev, n_keep=N_KEEP, m_group=M_GROUP):
+    Latent weights, codes and intermediates are shared; the step's inputs (X, dY) and
+    outputs (y, grad_X) come in ``n_io`` sets so that copies of one step can overlap
+    the compute of another."""
+
+    INPUTS = ["x_in", "x_down"] + [f"dy_{n}" for n, _, _ in LINEARS]
+
+    def __init__(self, host, dev, n_keep=N_KEEP, m_group=M_GROUP, n_io=1):
         import torch
 
         import sparsity_step_b200 as B
@@ -165,11 +171,16 @@ class Step:
         self.B = B
         self.n_keep, self.m_group = n_keep, m_group
         bf = torch.bfloat16
-        self.d = {}
-        for k, v in host.items():
-            t = v.to(dev, non_blocking=False)
-            self.d[k] = t.view(bf) if v.dtype == torch.int16 else t
         T = TOKENS
+        self.w = {n: host[f"w_{n}"].to(dev) for n, _, _ in LINEARS}
+        self.io = []
+        for _ in range(n_io):
+            d = {k: host[k].to(dev).view(bf) for k in self.INPUTS}
+            self.io.append({
+                "d": d,
+                "y": {n: torch.empty((T, n_out), dtype=bf, device=dev) for n, _, n_out in LINEARS},
+                "gx": {n: torch.empty((T, k_in), dtype=bf, device=dev) for n, k_in, _ in LINEARS},
+            })
         self.qm = {}
         self.ws_qm = {}
         for name, k_in, n_out in LINEARS:
@@ -185,19 +196,19 @@ class Step:
         self.a_in = torch.empty((T,), dtype=torch.float32, device=dev)
         self.xq_down = torch.empty((T, 11008), dtype=torch.int8, device=dev)
         self.a_down = torch.empty((T,), dtype=torch.float32, device=dev)
-        self.y = {n: torch.empty((T, n_out), dtype=bf, device=dev) for n, _, n_out in LINEARS}
-        self.gx = {n: torch.empty((T, k_in), dtype=bf, device=dev) for n, k_in, _ in LINEARS}
         self.gw = {n: torch.empty((n_out, k_in), dtype=bf, device=dev) for n, k_in, n_out in LINEARS}
         wsb = max(B.bitlinear_bwd_workspace_size(T, k, n, True) for _, k, n in LINEARS)
         self.ws_bwd = torch.empty((wsb,), dtype=torch.uint8, device=dev)
         self.launches_per_step = 3 * 3 + 2 + 3 + 3 * 3
 
-    def run(self, ev=None):
-        """Enqueue one step. ``ev`` maps a kernel class to a list that receives
-        (start, end) CUDA events around each of its launches."""
+    def run(self, ev=None, io=0):
+        """Enqueue one step on the current stream using I/O set ``io``. ``ev`` maps a
+        kernel class to a list that receives (start, end) CUDA events around each of
+        its launches."""
         import torch
 
         B = self.B
+        d, y, gx = self.io[io]["d"], self.io[io]["y"], self.io[io]["gx"]
 
         def timed(key, fn):
             if ev is None:
@@ -211,28 +222,77 @@ class Step:
 
         for name, _, _ in LINEARS:
             q = self.qm[name]
-            timed("quant_mask", lambda: B.bitlinear_quant_mask(self.d[f"w_{name}"], self.n_keep, self.m_group, out=q,
+            timed("quant_mask", lambda: B.bitlinear_quant_mask(self.w[name], self.n_keep, self.m_group, out=q,
                                                                workspace=self.ws_qm[name]))
-        timed("act_quant", lambda: B.bitlinear_act_quant(self.d["x_in"], xq=self.xq_in, absmax=self.a_in))
-        timed("act_quant", lambda: B.bitlinear_act_quant(self.d["x_down"], xq=self.xq_down, absmax=self.a_down))
+        timed("act_quant", lambda: B.bitlinear_act_quant(d["x_in"], xq=self.xq_in, absmax=self.a_in))
+        timed("act_quant", lambda: B.bitlinear_act_quant(d["x_down"], xq=self.xq_down, absmax=self.a_down))
         for name, _, _ in LINEARS:
             xq, a = (self.xq_down, self.a_down) if name == "down" else (self.xq_in, self.a_in)
             q = self.qm[name]
-            timed("fwd_i8_gemm", lambda: B.bitlinear_fwd(xq, a, q["w_scale"], w_i8=q["w_i8"], y=self.y[name]))
+            timed("fwd_i8_gemm", lambda: B.bitlinear_fwd(xq, a, q["w_scale"], w_i8=q["w_i8"], y=y[name]))
         for name, k_in, _ in LINEARS:
-            x = self.d["x_down"] if name == "down" else self.d["x_in"]
+            x = d["x_down"] if name == "down" else d["x_in"]
             q = self.qm[name]
-            dy = self.d[f"dy_{name}"]
+            dy = d[f"dy_{name}"]
             timed("bwd_grad_x", lambda: B.bitlinear_bwd(dy, None, q["codes"], q["w_scale"], want_grad_w=False,
-                                                        grad_x=self.gx[name], workspace=self.ws_bwd, k_in=k_in))
+                                                        grad_x=gx[name], workspace=self.ws_bwd, k_in=k_in))
             timed("bwd_grad_w", lambda: B.bitlinear_bwd(dy, x, None, None, want_grad_x=False, grad_w=self.gw[name]))
 
-    # bytes moved per step by the end-to-end variant
-    def e2e_inputs(self):
-        return ["x_in", "x_down"] + [f"dy_{n}" for n, _, _ in LINEARS]
+    def outputs(self, io=0):
+        return [self.io[io]["y"][n] for n, _, _ in LINEARS] + [self.io[io]["gx"][n] for n, _, _ in LINEARS]
 
-    def e2e_outputs(self):
-        return [self.y[n] for n, _, _ in LINEARS] + [self.gx[n] for n, _, _ in LINEARS]
+
+def run_e2e(step, host, steps, warmup, barrier):
+    """End-to-end steps through the public API: each step copies its inputs from
+    pinned host memory, runs, and copies its outputs back to pinned host memory.
+    Copies run on their own streams (host->device and device->host use separate copy
+    engines) and overlap the compute of the neighbouring steps through two I/O sets.
+    Returns (ms per step, h2d bytes per step, d2h bytes per step)."""
+    import torch
+
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    outs_host = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in step.outputs(0)] for _ in range(2)]
+    h2d = sum(host[k].numel() * host[k].element_size() for k in Step.INPUTS)
+    d2h = sum(t.numel() * t.element_size() for t in outs_host[0])
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_done + ev_out:
+        e.record(comp)
+
+    def one(i):
+        s = i % 2
+        io = step.io[s]
+        s_in.wait_event(ev_done[s])            # compute two steps back is done with this input set
+        with torch.cuda.stream(s_in):
+            for k in Step.INPUTS:
+                io["d"][k].view(torch.int16).copy_(host[k], non_blocking=True)
+        ev_in[s].record(s_in)
+        comp.wait_event(ev_in[s])
+        comp.wait_event(ev_out[s])             # this output set has been copied out
+        step.run(io=s)
+        ev_done[s].record(comp)
+        s_out.wait_event(ev_done[s])
+        with torch.cuda.stream(s_out):
+            for hdst, dsrc in zip(outs_host[s], step.outputs(s)):
+                hdst.copy_(dsrc, non_blocking=True)
+        ev_out[s].record(s_out)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize()
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(comp)
+    s_in.wait_event(t0)
+    for i in range(steps):
+        one(warmup + i)
+    comp.wait_event(ev_out[(warmup + steps - 1) % 2])
+    t1.record(comp)
+    torch.cuda.synchronize()
+    barrier()
+    return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
 def algorithmic_counts():
@@ -256,7 +316,7 @@ def run_ours(args) -> None:
     dev = torch.device("cuda", local)
 
     host = make_inputs(rank)
-    step = Step(host, dev)
+    step = Step(host, dev, n_io=2)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -318,29 +378,8 @@ def run_ours(args) -> None:
 
     # ---------------- end to end: pinned host inputs -> device -> step -> host outputs
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
-    outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in step.e2e_outputs()]
-    h2d = sum(host[k].numel() * host[k].element_size() for k in step.e2e_inputs())
-    d2h = sum(t.numel() * t.element_size() for t in outs_host)
-
-    def e2e_step():
-        for k in step.e2e_inputs():
-            step.d[k].view(torch.int16).copy_(host[k], non_blocking=True)
-        step.run()
-        for hdst, dsrc in zip(outs_host, step.e2e_outputs()):
-            hdst.copy_(dsrc, non_blocking=True)
-
-    for _ in range(min(args.warmup, 3)):
-        e2e_step()
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    ms_e2e, h2d, d2h = run_e2e(step, host, e2e_steps, min(args.warmup, 3), barrier)
+    ms_e2e = max_over_ranks(ms_e2e)
 
     # ---------------- raw tensor-pipe rates of this GPU (probe: MMAs from shared memory only)
     try:
@@ -392,7 +431,8 @@ def run_ours(args) -> None:
         "ms_per_step_8_8": round(ms_dense, 4),
         "roofline": roof,
         "e2e": {"value": round(TOKENS * world / (ms_e2e * 1e-3), 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 3), "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 3), "steps": e2e_steps,
+                "copies": "pinned host <-> device on separate H2D / D2H streams, overlapped with compute (2 I/O sets)"},
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -574,6 +614,119 @@ def run_case(args) -> None:
                       "rate": round(rate, 1), "unit": unit}), flush=True)
 
 
+DECODE_LAYERS = 36
+DECODE_SHAPES = [("q", 2048, 2048, "attn_in"), ("k", 2048, 256, "attn_in"), ("v", 2048, 256, "attn_in"),
+                 ("o", 2048, 2048, "o_in"), ("gate", 2048, 11008, "mlp_in"), ("up", 2048, 11008, "mlp_in"),
+                 ("down", 11008, 2048, "down_in")]
+DECODE_INPUTS = {"attn_in": 2048, "o_in": 2048, "mlp_in": 2048, "down_in": 11008}
+
+
+def run_decode(args) -> None:
+    """Qwen2.5-3B-shaped 36-layer stack of BitLinear layers (6:8), forward only:
+    decode steps at batch 1/8/32/128 (one grouped launch streams every layer's 2-bit
+    codes; the four per-shape inputs are reused across layers) and an 8192-token
+    prefill (tensor-core product per linear). Prints one JSON line."""
+    import numpy as np
+    import torch
+
+    import sparsity_step_b200 as B
+    from sparsity_step_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    layers = []   # per layer: {name: qm dict}
+    code_bytes = 0
+    n_keep, m_group = (8, 8) if args.dense else (N_KEEP, M_GROUP)
+    for layer in range(DECODE_LAYERS):
+        qms = {}
+        for i, (name, k_in, n_out, _) in enumerate(DECODE_SHAPES):
+            w = torch.from_numpy(synth.latent_weight(synth.config_seed(5, 100 * layer + i), n_out, k_in)).to(dev)
+            qms[name] = B.bitlinear_quant_mask(w, n_keep, m_group, want_mask=False, want_w_i8=args.prefill > 0)
+            qms[name].pop("workspace")
+            code_bytes += n_out * k_in // 4
+            del w
+        layers.append(qms)
+    torch.cuda.synchronize()
+
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    res = {"workload": "Qwen2.5-3B-shaped 36-layer BitLinear stack, forward",
+           "nm": f"{n_keep}:{m_group}", "code_bytes_per_step": code_bytes,
+           "hbm_peak_gbs": peaks["hbm_gbs"], "decode": {}}
+    for b in args.batches:
+        inputs = {k: bf(synth.activation_bf16(synth.config_seed(5, 9000 + kk), b, K, outliers=False))
+                  for kk, (k, K) in enumerate(DECODE_INPUTS.items())}
+        q = {k: B.bitlinear_act_quant(v) for k, v in inputs.items()}
+        probs = []
+        for qms in layers:
+            for name, k_in, n_out, src in DECODE_SHAPES:
+                xq, a = q[src]
+                probs.append({"xq": xq, "absmax": a, "codes": qms[name]["codes"], "w_scale": qms[name]["w_scale"],
+                              "y": torch.empty((b, n_out), dtype=torch.bfloat16, device=dev)})
+
+        def step():
+            for k, v in inputs.items():
+                B.bitlinear_act_quant(v, xq=q[k][0], absmax=q[k][1])
+            for s0 in range(0, len(probs), 256):
+                B.bitlinear_fwd_grouped(probs[s0:s0 + 256])
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        # one decode step is 5 short launches: replay it as a CUDA graph so that host
+        # launch overhead does not pace the GPU
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            graph.replay()
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / args.steps
+        del graph
+        act_bytes = sum(b * K * 3 + 4 * b for K in DECODE_INPUTS.values())   # bf16 read + int8 write + absmax
+        fwd_bytes = code_bytes + sum(b * k * 1 + 2 * b * n for _, k, n, _ in DECODE_SHAPES) * DECODE_LAYERS
+        gbs = (fwd_bytes + act_bytes) / (ms * 1e-3) / 1e9
+        res["decode"][f"b{b}"] = {"ms_per_step": round(ms, 4), "tok_s": round(b / (ms * 1e-3), 1),
+                                  "gb_s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                  "launches_per_step": len(DECODE_INPUTS) + (len(probs) + 255) // 256,
+                                  "cuda_graph": True}
+    if args.prefill > 0:
+        t = args.prefill
+        inputs = {k: bf(synth.activation_bf16(synth.config_seed(5, 9100 + kk), t, K, outliers=False))
+                  for kk, (k, K) in enumerate(DECODE_INPUTS.items())}
+        q = {k: B.bitlinear_act_quant(v) for k, v in inputs.items()}
+        ys = {name: torch.empty((t, n_out), dtype=torch.bfloat16, device=dev) for name, _, n_out, _ in DECODE_SHAPES}
+
+        def pstep():
+            for k, v in inputs.items():
+                B.bitlinear_act_quant(v, xq=q[k][0], absmax=q[k][1])
+            for qms in layers:
+                for name, k_in, n_out, src in DECODE_SHAPES:
+                    xq, a = q[src]
+                    B.bitlinear_fwd(xq, a, qms[name]["w_scale"], w_i8=qms[name]["w_i8"], y=ys[name])
+
+        pstep()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(max(1, args.steps // 10)):
+            pstep()
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / max(1, args.steps // 10)
+        ops = 2.0 * t * sum(k * n for _, k, n, _ in DECODE_SHAPES) * DECODE_LAYERS
+        res["prefill"] = {"tokens": t, "ms": round(ms, 3), "tok_s": round(t / (ms * 1e-3), 1),
+                          "tops_dense_equiv": round(ops / (ms * 1e-3) / 1e12, 1)}
+    print(json.dumps(res), flush=True)
+
+
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -591,7 +744,15 @@ def main(argv=None) -> None:
     ap.add_argument("--case-t", type=int, default=TOKENS)
     ap.add_argument("--case-k", type=int, default=2048)
     ap.add_argument("--case-n", type=int, default=11008)
+    ap.add_argument("--workload", choices=["train", "decode"], default="train",
+                    help="decode: the 36-layer stack at decode batches and prefill (separate JSON line)")
+    ap.add_argument("--batches", type=int, nargs="+", default=[1, 8, 32, 128])
+    ap.add_argument("--prefill", type=int, default=8192, help="prefill tokens for --workload decode (0 = skip)")
+    ap.add_argument("--dense", action="store_true", help="--workload decode with 8:8 (no mask)")
     args = ap.parse_args(argv)
+    if args.workload == "decode":
+        run_decode(args)
+        return
     if args.case:
         run_case(args)
         return

@@ -134,8 +134,8 @@ bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t
  *   xq [t, k_in] int8, absmax [t] fp32 (from bitlinear_act_quant).
  *   codes [n_out, k_in / 4] (packed masked codes), w_i8 [n_out, k_in] int8 (masked
  *   codes): give at least one. With w_i8 the product runs on the tcgen05 int8 tensor
- *   cores; with codes only it runs on a CUDA-core kernel that streams the 2-bit codes
- *   (meant for short decode batches).
+ *   cores (TMA-fed, for prefill and training shapes); with codes only it streams the
+ *   2-bit codes and decodes them into register MMA fragments (for decode batches).
  *   w_scale [1] fp32 gamma. acc_out [t, n_out] int32, out, nullable.
  *   y_out [t, n_out], out, bf16 (y_dtype = BL_OUT_BF16) or fp32 (BL_OUT_F32).
  * No bias term.
@@ -143,6 +143,28 @@ bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t
 bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* codes, const int8_t* w_i8,
                         const float* w_scale, int64_t t, int64_t k_in, int64_t n_out, int32_t* acc_out, void* y_out,
                         int y_dtype, void* stream);
+
+/* One forward problem of bitlinear_fwd_grouped (same meaning as the arguments of
+ * bitlinear_fwd, codes operand only). */
+typedef struct {
+  const int8_t* xq;       /* [t, k_in] int8 activations            */
+  const float* absmax;    /* [t] per-token absmax                   */
+  const uint8_t* codes;   /* [n_out, k_in / 4] packed masked codes  */
+  const float* w_scale;   /* [1] gamma                              */
+  int64_t t, k_in, n_out;
+  int32_t* acc_out;       /* [t, n_out] int32, nullable             */
+  void* y_out;            /* [t, n_out] bf16 or fp32                */
+} bl_fwd_problem;
+
+/*
+ * Step a4 for up to 256 independent problems in one launch (e.g. every BitLinear of
+ * a layer stack at one decode step, or the q/k/v or gate/up linears that share an
+ * input). Same result as bitlinear_fwd with the codes operand for each problem; the
+ * packed 2-bit codes are streamed once per 32 tokens. `problems` is a HOST array
+ * (copied into the launch); y_dtype applies to all problems. Problems may have t = 0.
+ * More than 256 problems: BL_ERR_UNSUPPORTED_SHAPE.
+ */
+bl_status bitlinear_fwd_grouped(const bl_fwd_problem* problems, int count, int y_dtype, void* stream);
 
 /* Bytes of workspace bitlinear_bwd needs (0 when grad_x is not requested). */
 size_t bitlinear_bwd_workspace_size(int64_t t, int64_t k_in, int64_t n_out, int want_grad_x);

@@ -12,6 +12,7 @@ from .bitlinear import (  # noqa: F401
     bitlinear_bwd_workspace_size,
     bitlinear_device_status,
     bitlinear_fwd,
+    bitlinear_fwd_grouped,
     bitlinear_quant_mask,
     bitlinear_quant_mask_noalloc,
     bitlinear_quant_mask_status,

@@ -27,6 +27,13 @@ _I64 = _c.c_int64
 _INT = _c.c_int
 _SZ = _c.c_size_t
 
+class BlFwdProblem(ctypes.Structure):
+    """bl_fwd_problem of include/bitlinear.h."""
+    _fields_ = [("xq", ctypes.c_void_p), ("absmax", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("w_scale", ctypes.c_void_p), ("t", ctypes.c_int64), ("k_in", ctypes.c_int64),
+                ("n_out", ctypes.c_int64), ("acc_out", ctypes.c_void_p), ("y_out", ctypes.c_void_p)]
+
+
 # name -> (restype, argtypes), in the order of include/bitlinear.h
 SIGNATURES = {
     "bitlinear_quant_mask_workspace_size": (_SZ, [_I64, _I64]),
@@ -35,6 +42,7 @@ SIGNATURES = {
     "bitlinear_quant_mask_noalloc": (_INT, [_P, _I64, _I64, _INT, _INT, _P, _P, _P, _P, _P]),
     "bitlinear_act_quant": (_INT, [_P, _I64, _I64, _P, _P, _P]),
     "bitlinear_fwd": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P]),
+    "bitlinear_fwd_grouped": (_INT, [_c.POINTER(BlFwdProblem), _INT, _INT, _P]),
     "bitlinear_bwd_workspace_size": (_SZ, [_I64, _I64, _I64, _INT]),
     "bitlinear_bwd": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _SZ, _P]),
     "bitlinear_device_status": (_INT, [_c.POINTER(_c.c_uint)]),

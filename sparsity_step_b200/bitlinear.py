@@ -127,6 +127,34 @@ def bitlinear_fwd(xq: torch.Tensor, absmax: torch.Tensor, w_scale: torch.Tensor,
     return y, acc
 
 
+def bitlinear_fwd_grouped(problems: list[dict], *, y_dtype=torch.bfloat16, stream=None) -> list[dict]:
+    """Forward product of several independent problems in one launch (codes operand).
+
+    Each problem is a dict with ``xq``, ``absmax``, ``codes``, ``w_scale`` and
+    optionally ``y``, ``acc`` (outputs allocated here when missing, ``want_acc`` to
+    request the int32 accumulators). Returns the dicts with ``y`` (and ``acc``) set.
+    """
+    arr = (_lib.BlFwdProblem * max(1, len(problems)))()
+    out = []
+    for i, p in enumerate(problems):
+        xq, codes = p["xq"], p["codes"]
+        t, k_in = xq.shape
+        n_out = codes.shape[0]
+        y = p.get("y")
+        if y is None:
+            y = torch.empty((t, n_out), dtype=y_dtype, device=xq.device)
+        acc = p.get("acc")
+        if acc is None and p.get("want_acc"):
+            acc = torch.empty((t, n_out), dtype=torch.int32, device=xq.device)
+        arr[i] = _lib.BlFwdProblem(_ptr(xq), _ptr(p["absmax"]), _ptr(codes), _ptr(p["w_scale"]), t, k_in, n_out,
+                                   _ptr(acc), _ptr(y))
+        out.append({**p, "y": y, "acc": acc})
+    ydt = BL_OUT_F32 if y_dtype == torch.float32 else BL_OUT_BF16
+    st = lib().bitlinear_fwd_grouped(arr, len(problems), ydt, _stream(stream))
+    check(st, "bitlinear_fwd_grouped")
+    return out
+
+
 def bitlinear_bwd_workspace_size(t: int, k_in: int, n_out: int, want_grad_x: bool = True) -> int:
     return int(lib().bitlinear_bwd_workspace_size(t, k_in, n_out, int(want_grad_x)))
 
@@ -170,6 +198,6 @@ def bitlinear_abi_version() -> int:
 __all__ = [
     "bitlinear_quant_mask_workspace_size", "bitlinear_quant_mask", "bitlinear_quant_mask_status",
     "bitlinear_quant_mask_noalloc",
-    "bitlinear_act_quant", "bitlinear_fwd", "bitlinear_bwd_workspace_size", "bitlinear_bwd",
+    "bitlinear_act_quant", "bitlinear_fwd", "bitlinear_fwd_grouped", "bitlinear_bwd_workspace_size", "bitlinear_bwd",
     "bitlinear_device_status", "bitlinear_abi_version", "BL_OUT_BF16", "BL_OUT_F32", "_lib",
 ]

@@ -108,6 +108,60 @@ bl_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
   return BL_OK;
 }
 
+// ------------------------------------------------------------------ grouped codes product
+
+template <int NG>
+bl_status launch_fwd_codes_ng(const bl::FwdGroup& grp, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(bl::fwd_codes_mma_kernel<NG>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+    attr_set = true;
+  }
+  const int warps_per_block = bl::kDecodeThreads / 32;
+  int64_t blocks = (static_cast<int64_t>(grp.total_tasks) + warps_per_block - 1) / warps_per_block;
+  const int64_t cap = int64_t(device_sm_count()) * 4;
+  if (blocks > cap) blocks = cap;
+  bl::fwd_codes_mma_kernel<NG><<<static_cast<unsigned>(blocks), bl::kDecodeThreads, 0, st>>>(grp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return BL_OK;
+}
+
+// Problems are already validated. Builds the task table in kernel parameters.
+bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32, cudaStream_t st) {
+  int64_t tmax = 0;
+  for (int i = 0; i < count; ++i) tmax = problems[i].t > tmax ? problems[i].t : tmax;
+  if (tmax == 0) return BL_OK;
+  const int ng = tmax <= 8 ? 1 : (tmax <= 16 ? 2 : 4);
+  static thread_local bl::FwdGroup grp;   // ~16 KB: kept off the stack
+  int64_t tasks = 0;
+  int n = 0;
+  for (int i = 0; i < count; ++i) {
+    const bl_fwd_problem& q = problems[i];
+    if (q.t == 0) continue;
+    bl::FwdProblem& d = grp.p[n++];
+    d.codes = q.codes;
+    d.xq = q.xq;
+    d.absmax = q.absmax;
+    d.w_scale = q.w_scale;
+    d.y = q.y_out;
+    d.acc = q.acc_out;
+    d.t = static_cast<int>(q.t);
+    d.k_in = static_cast<int>(q.k_in);
+    d.n_out = static_cast<int>(q.n_out);
+    d.task_begin = static_cast<int>(tasks);
+    tasks += (q.n_out / 16) * ((q.t + 8 * ng - 1) / (8 * ng));
+    if (tasks > INT32_MAX) return fail(BL_ERR_UNSUPPORTED_SHAPE, "too much work in one call");
+  }
+  grp.count = n;
+  grp.total_tasks = static_cast<int>(tasks);
+  grp.y_f32 = y_f32 ? 1 : 0;
+  if (ng == 1) return launch_fwd_codes_ng<1>(grp, st);
+  if (ng == 2) return launch_fwd_codes_ng<2>(grp, st);
+  return launch_fwd_codes_ng<4>(grp, st);
+}
+
 // ------------------------------------------------------------------ quant_mask sizing
 
 constexpr int kQmTargetBlocks = 148 * 8;
@@ -259,13 +313,25 @@ bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* co
     if (bl_status s = make_out_map(&to, y_out, t, n_out, g.out_f32)) return s;
     return launch_gemm<true, false, false, bl::EPI_FWD, true>(ta, tb, to, g, st);
   }
-  const unsigned grid = static_cast<unsigned>((n_out + bl::kCodesWarps - 1) / bl::kCodesWarps);
-  bl::fwd_codes_kernel<<<grid, bl::kCodesWarps * 32, 0, st>>>(xq, absmax, codes, w_scale, static_cast<int>(t),
-                                                              static_cast<int>(k_in), static_cast<int>(n_out), acc_out,
-                                                              y_out, y_dtype == BL_OUT_F32);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "fwd_codes launch");
-  return BL_OK;
+  bl_fwd_problem prob{xq, absmax, codes, w_scale, t, k_in, n_out, acc_out, y_out};
+  return launch_fwd_codes(&prob, 1, y_dtype == BL_OUT_F32, st);
+}
+
+bl_status bitlinear_fwd_grouped(const bl_fwd_problem* problems, int count, int y_dtype, void* stream) {
+  g_err[0] = 0;
+  if (!problems || count < 0) return fail(BL_ERR_INVALID_ARG, "problems is required");
+  if (count > bl::kMaxFwdGroup) return fail(BL_ERR_UNSUPPORTED_SHAPE, "at most %d problems per call", bl::kMaxFwdGroup);
+  if (y_dtype != BL_OUT_BF16 && y_dtype != BL_OUT_F32) return fail(BL_ERR_INVALID_ARG, "y_dtype must be BL_OUT_BF16 or BL_OUT_F32");
+  for (int i = 0; i < count; ++i) {
+    const bl_fwd_problem& q = problems[i];
+    if (bl_status s = check_shape(q.t, q.k_in, q.n_out)) return fail(s, "problem %d: %s", i, g_err);
+    if (!q.codes || !q.w_scale) return fail(BL_ERR_INVALID_ARG, "problem %d: codes and w_scale are required", i);
+    if (q.t > 0 && (!q.xq || !q.absmax || !q.y_out)) return fail(BL_ERR_INVALID_ARG, "problem %d: xq, absmax, y_out are required", i);
+    if (!aligned16(q.codes) || !aligned16(q.w_scale) || (q.xq && !aligned16(q.xq)) || (q.absmax && !aligned16(q.absmax)) ||
+        (q.y_out && !aligned16(q.y_out)) || (q.acc_out && !aligned16(q.acc_out)))
+      return fail(BL_ERR_ALIGNMENT, "problem %d: every pointer must be 16-byte aligned", i);
+  }
+  return launch_fwd_codes(problems, count, y_dtype == BL_OUT_F32, as_stream(stream));
 }
 
 size_t bitlinear_bwd_workspace_size(int64_t t, int64_t k_in, int64_t n_out, int want_grad_x) {

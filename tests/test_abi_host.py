@@ -82,6 +82,28 @@ def test_fwd_validation(L):
     del args
 
 
+def test_fwd_grouped_validation(L):
+    P = _lib.BlFwdProblem
+    arr = (P * 2)(P(GOOD, GOOD, GOOD, GOOD, 4, 896, 896, None, GOOD), P(GOOD, GOOD, GOOD, GOOD, 1, 2048, 256, None, GOOD))
+    assert L.bitlinear_fwd_grouped(None, 1, 0, None) == -1
+    assert L.bitlinear_fwd_grouped(arr, 257, 0, None) == -2
+    assert L.bitlinear_fwd_grouped(arr, 2, 5, None) == -1
+    arr[1].k_in = 100
+    assert L.bitlinear_fwd_grouped(arr, 2, 0, None) == -2
+    assert "problem 1" in _err(L)
+    arr[1].k_in = 2048
+    arr[1].codes = None
+    assert L.bitlinear_fwd_grouped(arr, 2, 0, None) == -1
+    arr[1].codes = BAD
+    assert L.bitlinear_fwd_grouped(arr, 2, 0, None) == -3
+    # empty problems enqueue nothing
+    arr[0].t = 0
+    arr[1].t = 0
+    arr[1].codes = GOOD
+    assert L.bitlinear_fwd_grouped(arr, 2, 0, None) == 0
+    assert L.bitlinear_fwd_grouped(arr, 0, 0, None) == 0
+
+
 def test_bwd_validation(L):
     need = L.bitlinear_bwd_workspace_size(16, 896, 896, 1)
     assert need == 896 * 896 * 2

@@ -160,6 +160,26 @@ def test_config5_decode_batches(idx, layer):
                   f32=(b == 8))
 
 
+@pytest.mark.parametrize("b", [1, 3, 8, 16, 32, 128])
+def test_config5_grouped_layer(b):
+    """All seven linears of one layer in one grouped launch, mixed shapes."""
+    probs, refs = [], []
+    for idx, (_, k_in, n_out) in enumerate(QWEN3B_LAYER):
+        w = synth.latent_weight(synth.config_seed(5, 300 + idx), n_out, k_in)
+        x = synth.activation_bf16(synth.config_seed(5, 400 + idx + b), b, k_in, outliers=False)
+        ref_qm = O.quant_mask(w, 6, 8)
+        qm = gpu_quant_mask(w, 6, 8)
+        ref_q, ref_a = O.act_quant(x)
+        xq, a = gpu_act_quant(x)
+        probs.append({"xq": xq, "absmax": a, "codes": qm["codes"], "w_scale": qm["w_scale"], "want_acc": True})
+        refs.append(O.fwd(ref_q, ref_a, ref_qm["mcode"], ref_qm["gamma"]))
+    out = B.bitlinear_fwd_grouped(probs)
+    torch.cuda.synchronize()
+    for (acc_ref, y_ref), o, (name, _, _) in zip(refs, out, QWEN3B_LAYER):
+        assert_exact(o["acc"].cpu().numpy(), acc_ref, f"grouped b{b} {name} acc")
+        assert_bf16_within_ulp(bf16_dev_to_bits(o["y"]), y_ref, f"grouped b{b} {name} y")
+
+
 @pytest.mark.parametrize("idx", [0, 6], ids=["q", "down"])
 def test_config5_prefill_8192(idx):
     _, k_in, n_out = QWEN3B_LAYER[idx]
