@@ -3,11 +3,11 @@
 // BitNet b1.58 2B4T article (lsdiaocha.cn), section 一: activations are quantised
 // to 8-bit integers; section 四: W1.58A8 (ternary weights x int8 activations).
 //
-// One CTA per token row. Each thread loads its 16-byte vectors of the row once and
-// keeps them in registers; the row absmax is a block max over |bf16| bit patterns
-// (exact, order-free); then q = clamp(rint(x * (127 / a)), -128, 127) with one
-// IEEE fp32 division per row and one fp32 multiply per element (no FMA), and the
-// int8 row is written with 8-byte stores. HBM traffic: 2 B read + 1 B written per
+// Each CTA handles R token rows. Each thread loads its 16-byte vectors of the rows
+// once and keeps them in registers; a row's absmax is a block max over |bf16| bit
+// patterns (exact, order-free); then q = clamp(rint(x * (127 / a)), -128, 127) with
+// one IEEE fp32 division per row and one fp32 multiply per element (no FMA), and the
+// int8 rows are written with 8-byte stores. HBM traffic: 2 B read + 1 B written per
 // element, + 4 B per row.
 #pragma once
 
@@ -44,37 +44,94 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t m, uint32_t* s_red) {
   return r;
 }
 
-// Row cached in registers: VPT 16-byte vectors (8 bf16 each) per thread.
-template <int VPT>
-__global__ void __launch_bounds__(256) act_quant_kernel(const uint4* __restrict__ x, int k8, int8_t* __restrict__ xq,
+// R rows per CTA, each cached in registers: VPT 16-byte vectors (8 bf16) per thread
+// per row. All R rows' loads are in flight before one block reduction of R maxima.
+template <int VPT, int R>
+__global__ void __launch_bounds__(256) act_quant_kernel(const uint4* __restrict__ x, int64_t t, int k8, int8_t* __restrict__ xq,
                                                         float* __restrict__ absmax_out) {
-  __shared__ uint32_t s_red[8];
-  const int64_t row = blockIdx.x;
-  const uint4* xr = x + row * k8;
-  uint4 v[VPT];
-  uint32_t m = 0;
+  __shared__ uint32_t s_red[R][8];
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * R;
+  uint4 v[R][VPT];
+  uint32_t m[R];
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int idx = threadIdx.x + i * blockDim.x;
-    if (idx < k8) {
-      v[i] = __ldcs(xr + idx);
-      m = bf16x2_absmax(v[i].x, m);
-      m = bf16x2_absmax(v[i].y, m);
-      m = bf16x2_absmax(v[i].z, m);
-      m = bf16x2_absmax(v[i].w, m);
+  for (int r = 0; r < R; ++r) {
+    m[r] = 0;
+    const bool row_ok = row0 + r < t;
+    const uint4* xr = x + (row0 + r) * k8;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = threadIdx.x + i * blockDim.x;
+      if (row_ok && idx < k8) {
+        v[r][i] = __ldcs(xr + idx);
+        m[r] = bf16x2_absmax(v[r][i].x, m[r]);
+        m[r] = bf16x2_absmax(v[r][i].y, m[r]);
+        m[r] = bf16x2_absmax(v[r][i].z, m[r]);
+        m[r] = bf16x2_absmax(v[r][i].w, m[r]);
+      }
     }
   }
-  m = block_max_u32(m, s_red);
-  float a = __uint_as_float(m << 16);
-  if (a == 0.0f) a = 1e-5f;   // an all-zero row quantises to zeros
-  const float s = __fdiv_rn(127.0f, a);
-  uint2* out = reinterpret_cast<uint2*>(xq + row * (static_cast<int64_t>(k8) * 8));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int idx = threadIdx.x + i * blockDim.x;
-    if (idx < k8) out[idx] = make_uint2(quant_pack4(v[i].x, v[i].y, s), quant_pack4(v[i].z, v[i].w, s));
+  for (int r = 0; r < R; ++r) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m[r] = max(m[r], __shfl_xor_sync(0xffffffffu, m[r], off));
+    if (lane == 0) s_red[r][warp] = m[r];
   }
-  if (threadIdx.x == 0) absmax_out[row] = a;
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (row0 + r >= t) break;
+    uint32_t mm = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) mm = max(mm, s_red[r][w]);
+    float a = __uint_as_float(mm << 16);
+    if (a == 0.0f) a = 1e-5f;   // an all-zero row quantises to zeros
+    const float sc = __fdiv_rn(127.0f, a);
+    uint2* out = reinterpret_cast<uint2*>(xq + (row0 + r) * (static_cast<int64_t>(k8) * 8));
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = threadIdx.x + i * blockDim.x;
+      if (idx < k8) out[idx] = make_uint2(quant_pack4(v[r][i].x, v[r][i].y, sc), quant_pack4(v[r][i].z, v[r][i].w, sc));
+    }
+    if (threadIdx.x == 0) absmax_out[row0 + r] = a;
+  }
+}
+
+// Short rows (k8 <= 32 * VPT): one warp per row, the row held in registers (VPT
+// 16-byte vectors per lane), warp-shuffle max, no block barrier. Persistent warps
+// stride over the rows.
+template <int VPT>
+__global__ void __launch_bounds__(256) act_quant_warp_kernel(const uint4* __restrict__ x, int64_t t, int k8,
+                                                             int8_t* __restrict__ xq, float* __restrict__ absmax_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < t; row += warps) {
+    const uint4* xr = x + row * k8;
+    uint4 v[VPT];
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = lane + 32 * i;
+      if (idx < k8) {
+        v[i] = __ldcs(xr + idx);
+        m = bf16x2_absmax(v[i].x, m);
+        m = bf16x2_absmax(v[i].y, m);
+        m = bf16x2_absmax(v[i].z, m);
+        m = bf16x2_absmax(v[i].w, m);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float a = __uint_as_float(m << 16);
+    if (a == 0.0f) a = 1e-5f;   // an all-zero row quantises to zeros
+    const float sc = __fdiv_rn(127.0f, a);
+    uint2* out = reinterpret_cast<uint2*>(xq + row * (static_cast<int64_t>(k8) * 8));
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = lane + 32 * i;
+      if (idx < k8) out[idx] = make_uint2(quant_pack4(v[i].x, v[i].y, sc), quant_pack4(v[i].z, v[i].w, sc));
+    }
+    if (lane == 0) absmax_out[row] = a;
+  }
 }
 
 // Rows too long to cache in registers: read the row twice (max, then quantise).

@@ -112,17 +112,18 @@ bl_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
 
 template <int NG>
 bl_status launch_fwd_codes_ng(const bl::FwdGroup& grp, cudaStream_t st) {
+  using C = bl::DecCfg<NG>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(bl::fwd_codes_mma_kernel<NG>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaError_t e = cudaFuncSetAttribute(bl::fwd_codes_mma_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
     attr_set = true;
   }
-  const int warps_per_block = bl::kDecodeThreads / 32;
-  int64_t blocks = (static_cast<int64_t>(grp.total_tasks) + warps_per_block - 1) / warps_per_block;
-  const int64_t cap = int64_t(device_sm_count()) * 4;
+  int64_t blocks = (static_cast<int64_t>(grp.total_tasks) + C::kWarps - 1) / C::kWarps;
+  const int64_t cap = int64_t(device_sm_count());   // one CTA per SM (persistent)
   if (blocks > cap) blocks = cap;
-  bl::fwd_codes_mma_kernel<NG><<<static_cast<unsigned>(blocks), bl::kDecodeThreads, 0, st>>>(grp);
+  bl::fwd_codes_mma_kernel<NG><<<static_cast<unsigned>(blocks), C::kThreads, C::kSmemBytes, st>>>(grp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return BL_OK;
@@ -160,6 +161,54 @@ bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32
   if (ng == 1) return launch_fwd_codes_ng<1>(grp, st);
   if (ng == 2) return launch_fwd_codes_ng<2>(grp, st);
   return launch_fwd_codes_ng<4>(grp, st);
+}
+
+// ------------------------------------------------------------------ quant_mask launches
+
+template <int M, int NK>
+void launch_mask_codes(const float* w, int64_t n8, int n_keep, const float* gamma, uint8_t* mask, uint8_t* codes,
+                       int8_t* w_i8, int grid, cudaStream_t st) {
+  bl::qm_mask_codes_kernel<M, NK><<<grid, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w), n8, n_keep, gamma,
+                                                                     mask, reinterpret_cast<uint16_t*>(codes),
+                                                                     reinterpret_cast<uint2*>(w_i8));
+}
+
+int qm_blocks(int64_t numel);
+
+// Both passes of steps a1 + a2 on `scratch` (its first 16 bytes are cleared here).
+bl_status enqueue_quant_mask(const float* w, int64_t n_out, int64_t k_in, int n_keep, int m_group, uint8_t* mask,
+                             uint8_t* codes, int8_t* w_i8, float* gamma, void* scratch, cudaStream_t st) {
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 16, st);   // range flag, status, blocks-done ticket
+  if (e != cudaSuccess) return cuda_fail(e, "scratch reset");
+  const int64_t numel = n_out * k_in;
+  const int blocks = qm_blocks(numel);
+  bl::QmScratch q{reinterpret_cast<unsigned int*>(ws), reinterpret_cast<int*>(ws + 4),
+                  reinterpret_cast<unsigned int*>(ws + 8), reinterpret_cast<unsigned long long*>(ws + bl::kQmWsHeader)};
+  bl::qm_abs_sum_kernel<<<blocks, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w), numel / 4, numel, q, gamma);
+  const int64_t n8 = numel / 8;
+  int64_t g2 = (n8 + bl::kQmThreads - 1) / bl::kQmThreads;
+  const int64_t cap = int64_t(device_sm_count()) * 16;
+  if (g2 > cap) g2 = cap;
+  const int grid = static_cast<int>(g2);
+  if (m_group == 8) {
+    switch (n_keep) {
+      case 8: launch_mask_codes<8, 8>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+      case 6: launch_mask_codes<8, 6>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+      case 4: launch_mask_codes<8, 4>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+      case 2: launch_mask_codes<8, 2>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+      default: launch_mask_codes<8, 0>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+    }
+  } else {
+    switch (n_keep) {
+      case 4: launch_mask_codes<4, 4>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+      case 2: launch_mask_codes<4, 2>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+      default: launch_mask_codes<4, 0>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+    }
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quant_mask launch");
+  return BL_OK;
 }
 
 // ------------------------------------------------------------------ quant_mask sizing
@@ -206,34 +255,8 @@ bl_status bitlinear_quant_mask(const float* w_latent, int64_t n_out, int64_t k_i
   if (!aligned16(w_latent) || !aligned16(codes_out) || !aligned16(w_scale_out) || !aligned16(workspace) ||
       (mask_out && !aligned16(mask_out)) || (w_i8_out && !aligned16(w_i8_out)))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
-  cudaStream_t st = as_stream(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  unsigned int* range_flag = reinterpret_cast<unsigned int*>(ws);
-  int* status = reinterpret_cast<int*>(ws + 4);
-  unsigned long long* partials = reinterpret_cast<unsigned long long*>(ws + bl::kQmWsHeader);
-  cudaError_t e = cudaMemsetAsync(ws, 0, 16, st);
-  if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
-  const int blocks = qm_blocks(numel);
-  bl::qm_abs_sum_kernel<<<blocks, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), numel / 4, partials,
-                                                          range_flag);
-  bl::qm_finalize_kernel<<<1, 256, 0, st>>>(partials, blocks, numel, range_flag, status, w_scale_out);
-  const int64_t n8 = numel / 8;
-  int64_t g2 = (n8 + bl::kQmThreads - 1) / bl::kQmThreads;
-  const int64_t cap = int64_t(device_sm_count()) * 16;
-  if (g2 > cap) g2 = cap;
-  if (m_group == 8)
-    bl::qm_mask_codes_kernel<8><<<(int)g2, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), n8, n_keep,
-                                                                     w_scale_out, mask_out,
-                                                                     reinterpret_cast<uint16_t*>(codes_out),
-                                                                     reinterpret_cast<uint2*>(w_i8_out));
-  else
-    bl::qm_mask_codes_kernel<4><<<(int)g2, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), n8, n_keep,
-                                                                     w_scale_out, mask_out,
-                                                                     reinterpret_cast<uint16_t*>(codes_out),
-                                                                     reinterpret_cast<uint2*>(w_i8_out));
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "quant_mask launch");
-  return BL_OK;
+  return enqueue_quant_mask(w_latent, n_out, k_in, n_keep, m_group, mask_out, codes_out, w_i8_out, w_scale_out,
+                            workspace, as_stream(stream));
 }
 
 bl_status bitlinear_quant_mask_status(const void* workspace, void* stream) {
@@ -258,18 +281,24 @@ bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t
   cudaStream_t st = as_stream(stream);
   const int k8 = static_cast<int>(k_in / 8);
   const uint4* xv = reinterpret_cast<const uint4*>(x);
-  const unsigned grid = static_cast<unsigned>(t);
-  if (k8 <= 128) {
-    bl::act_quant_kernel<1><<<grid, 128, 0, st>>>(xv, k8, xq_out, absmax_out);
-  } else {
+  const unsigned g1 = static_cast<unsigned>(t);
+  if (k8 <= 512) {   // k_in <= 4096: one warp per row
+    const int per_sm = k8 <= 128 ? 8 : (k8 <= 256 ? 4 : 2);   // resident 256-thread blocks (registers)
+    int64_t blocks = (t + 7) / 8;
+    const int64_t cap = int64_t(device_sm_count()) * per_sm;
+    if (blocks > cap) blocks = cap;
+    const unsigned gb = static_cast<unsigned>(blocks);
+    if (k8 <= 128) bl::act_quant_warp_kernel<4><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (k8 <= 256) bl::act_quant_warp_kernel<8><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else bl::act_quant_warp_kernel<16><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+  } else {   // one CTA per row
     const int vpt = (k8 + 255) / 256;
-    if (vpt <= 2) bl::act_quant_kernel<2><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
-    else if (vpt <= 4) bl::act_quant_kernel<4><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
-    else if (vpt <= 6) bl::act_quant_kernel<6><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
-    else if (vpt <= 8) bl::act_quant_kernel<8><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
-    else if (vpt <= 12) bl::act_quant_kernel<12><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
-    else if (vpt <= 16) bl::act_quant_kernel<16><<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
-    else bl::act_quant_long_kernel<<<grid, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+    if (vpt <= 4) bl::act_quant_kernel<4, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (vpt <= 6) bl::act_quant_kernel<6, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (vpt <= 8) bl::act_quant_kernel<8, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (vpt <= 12) bl::act_quant_kernel<12, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (vpt <= 16) bl::act_quant_kernel<16, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else bl::act_quant_long_kernel<<<g1, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
@@ -491,32 +520,6 @@ extern "C" bl_status bitlinear_quant_mask_noalloc(const float* w_latent, int64_t
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
   void* scratch = nullptr;
   if (bl_status s = noalloc_scratch(&scratch)) return s;
-  cudaStream_t st = as_stream(stream);
-  uint8_t* ws = static_cast<uint8_t*>(scratch);
-  unsigned int* range_flag = reinterpret_cast<unsigned int*>(ws);
-  int* status = reinterpret_cast<int*>(ws + 4);
-  unsigned long long* partials = reinterpret_cast<unsigned long long*>(ws + bl::kQmWsHeader);
-  cudaError_t e = cudaMemsetAsync(ws, 0, 16, st);   // range flag and status start at zero
-  if (e != cudaSuccess) return cuda_fail(e, "scratch reset");
-  const int blocks = qm_blocks(numel);
-  bl::qm_abs_sum_kernel<<<blocks, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), numel / 4, partials,
-                                                          range_flag);
-  bl::qm_finalize_kernel<<<1, 256, 0, st>>>(partials, blocks, numel, range_flag, status, w_scale_out);
-  const int64_t n8 = numel / 8;
-  int64_t g2 = (n8 + bl::kQmThreads - 1) / bl::kQmThreads;
-  const int64_t cap = int64_t(device_sm_count()) * 16;
-  if (g2 > cap) g2 = cap;
-  if (m_group == 8)
-    bl::qm_mask_codes_kernel<8><<<(int)g2, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), n8, n_keep,
-                                                                     w_scale_out, mask_out,
-                                                                     reinterpret_cast<uint16_t*>(codes_out),
-                                                                     reinterpret_cast<uint2*>(w_i8_out));
-  else
-    bl::qm_mask_codes_kernel<4><<<(int)g2, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w_latent), n8, n_keep,
-                                                                     w_scale_out, mask_out,
-                                                                     reinterpret_cast<uint16_t*>(codes_out),
-                                                                     reinterpret_cast<uint2*>(w_i8_out));
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "quant_mask_noalloc launch");
-  return BL_OK;
+  return enqueue_quant_mask(w_latent, n_out, k_in, n_keep, m_group, mask_out, codes_out, w_i8_out, w_scale_out, scratch,
+                            as_stream(stream));
 }

@@ -44,9 +44,10 @@ __global__ void __launch_bounds__(256) expand_codes_bf16_kernel(const uint32_t* 
 // decode step). Work is split into tasks of 16 weight rows x 32 tokens; persistent
 // warps stride over the concatenated task list.
 //
-// Per task a warp streams its 16 rows' codes once (16-byte loads, L1 bypass) and
+// Per task a warp streams its 16 rows' codes once (each thread prefetches its own 32
+// bytes per chunk with cp.async, kDecDepth chunks ahead across task boundaries) and
 // feeds mma.sync.m16n8k32.s8 with the weights decoded straight into A fragments in
-// registers: weights never pass through shared memory. Inside each chunk of 256
+// registers: decoded weights never pass through shared memory. Inside each chunk of 256
 // weights the reduction order is permuted so that thread (group g, index tig) owns
 // logical weights [64*tig, 64*tig + 64): MMA step s, A/B slot 4*tig + i holds weight
 // 64*tig + 8*s + i and slot 4*tig + 16 + i holds 64*tig + 8*s + 4 + i. A thread then
@@ -55,7 +56,6 @@ __global__ void __launch_bounds__(256) expand_codes_bf16_kernel(const uint32_t* 
 // Code bytes become int8x4 words through a 256-entry table replicated per lane
 // (entry e of lane l at word 32*e + l: conflict-free).
 constexpr int kMaxFwdGroup = 256;
-constexpr int kDecodeThreads = 256;
 
 struct FwdProblem {
   const uint8_t* codes;    // [n_out, k_in/4]
@@ -92,15 +92,108 @@ __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ uint32_t byte_of(const uint4& v, int i) {
-  const uint32_t w = i < 4 ? v.x : (i < 8 ? v.y : (i < 12 ? v.z : v.w));
-  return (w >> (8 * (i & 3))) & 0xFFu;
+// Table lookup of code byte j (0..3) of word w for this lane: entry e of lane l is the
+// 32-bit word at byte offset 128*e + 4*l of the table, so the offset is
+// ((w >> (8j - 7)) & 0x7F80) | 4*lane: one shift and one logic op, conflict-free.
+template <int J>
+__device__ __forceinline__ uint32_t lut_lookup(const uint32_t* lut, uint32_t w, uint32_t lane4) {
+  const uint32_t off = ((J == 0 ? (w << 7) : (w >> (8 * J - 7))) & 0x7F80u) | lane4;
+  return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(lut) + off);
 }
 
+// Accumulators per token group, optionally split into independent sets (summed at
+// the end) to shorten the MMA dependency chain; one set measured fastest because
+// the registers a split costs lower the number of resident warps.
+template <int NG>
+struct DecAcc {
+  static constexpr int kSets = 1;   // more sets did not help (they cost occupancy)
+  int v[kSets][NG][4];
+};
+
+// Two MMA steps from one 32-bit word of each row's codes (bytes 0..3 = steps 2h, 2h+1).
+template <int NG>
+__device__ __forceinline__ void decode_mma_word(DecAcc<NG>& acc, const uint32_t* lut, uint32_t lane4, uint32_t w0,
+                                                uint32_t w1, const uint4 (&xv)[NG][4], int h) {
+  constexpr int S = DecAcc<NG>::kSets;
+  {   // step 2h: bytes 0 (a0) and 1 (a2) of row g's word, of row g+8's word (a1, a3)
+    const uint32_t a0 = lut_lookup<0>(lut, w0, lane4), a2 = lut_lookup<1>(lut, w0, lane4);
+    const uint32_t a1 = lut_lookup<0>(lut, w1, lane4), a3 = lut_lookup<1>(lut, w1, lane4);
+#pragma unroll
+    for (int j = 0; j < NG; ++j) mma_m16n8k32_s8(acc.v[(2 * h) % S][j], a0, a1, a2, a3, xv[j][h].x, xv[j][h].y);
+  }
+  {   // step 2h+1: bytes 2, 3
+    const uint32_t a0 = lut_lookup<2>(lut, w0, lane4), a2 = lut_lookup<3>(lut, w0, lane4);
+    const uint32_t a1 = lut_lookup<2>(lut, w1, lane4), a3 = lut_lookup<3>(lut, w1, lane4);
+#pragma unroll
+    for (int j = 0; j < NG; ++j) mma_m16n8k32_s8(acc.v[(2 * h + 1) % S][j], a0, a1, a2, a3, xv[j][h].z, xv[j][h].w);
+  }
+}
+
+template <int NG>
+__device__ __forceinline__ void decode_chunk(DecAcc<NG>& acc, const uint32_t* lut, uint32_t lane4, const uint4& c0,
+                                             const uint4& c1, const uint4 (&xv)[NG][4]) {
+  decode_mma_word<NG>(acc, lut, lane4, c0.x, c1.x, xv, 0);
+  decode_mma_word<NG>(acc, lut, lane4, c0.y, c1.y, xv, 1);
+  decode_mma_word<NG>(acc, lut, lane4, c0.z, c1.z, xv, 2);
+  decode_mma_word<NG>(acc, lut, lane4, c0.w, c1.w, xv, 3);
+}
+
+// Per-thread streaming: each thread copies the 32 code bytes it will itself decode
+// per chunk (16 bytes of row g, 16 of row g+8) with cp.async into its own slots of a
+// shared-memory ring kDecDepth chunks deep, so up to kDecDepth chunks per warp are in
+// flight without holding registers, and no thread ever reads another thread's data.
+// Ring layout [chunk slot][row half][thread][16 B]: consecutive threads read
+// consecutive 16-byte slots (conflict-free).
+constexpr int kDecDepth = 4;
+constexpr int kDecLutBytes = 256 * 32 * 4;
+
+template <int NG>
+struct DecCfg {
+  static constexpr int kWarps = NG == 1 ? 32 : 16;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kRingBytes = kDecDepth * 2 * kThreads * 16;
+  static constexpr int kSmemBytes = kDecLutBytes + kRingBytes;
+};
+
+struct DecTask {
+  const FwdProblem* P;
+  int n0, t0, nch;   // first row, first token, chunks of 256 weights
+};
+
+__device__ __forceinline__ DecTask dec_task(const FwdGroup& G, int task, int tok_per_task) {
+  int lo = 0, hi = G.count - 1;   // last problem with task_begin <= task
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (G.p[mid].task_begin <= task) lo = mid;
+    else hi = mid - 1;
+  }
+  const FwdProblem& P = G.p[lo];
+  const int row_blocks = P.n_out >> 4;
+  const int local = task - P.task_begin;
+  DecTask d;
+  d.P = &P;
+  d.n0 = (local % row_blocks) * 16;
+  d.t0 = (local / row_blocks) * tok_per_task;
+  d.nch = (P.k_in + 255) >> 8;
+  return d;
+}
+
+// 16-byte async copy global -> shared; `valid` false writes zeros (src not read).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <int NG>   // token groups of 8 per task (1, 2 or 4)
-__global__ void __launch_bounds__(kDecodeThreads) fwd_codes_mma_kernel(const __grid_constant__ FwdGroup G) {
-  __shared__ uint32_t lut[256 * 32];
-  const int lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(const __grid_constant__ FwdGroup G) {
+  using C = DecCfg<NG>;
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  uint32_t* lut = reinterpret_cast<uint32_t*>(dsmem);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
     const uint32_t e = static_cast<uint32_t>(i) >> 5;
     uint32_t word = 0;
@@ -112,72 +205,94 @@ __global__ void __launch_bounds__(kDecodeThreads) fwd_codes_mma_kernel(const __g
     lut[i] = word;
   }
   __syncthreads();
-  const uint32_t* my_lut = lut + lane;
+  const uint32_t ring = smem_u32(dsmem + kDecLutBytes) + static_cast<uint32_t>(threadIdx.x * 16);
+  constexpr uint32_t kSlot = 2 * C::kThreads * 16;    // bytes per chunk slot
+  constexpr uint32_t kHalf = C::kThreads * 16;        // row g -> row g+8 within a slot
+
+  const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
   const int g = lane >> 2, tig = lane & 3;
-  const int warps = (gridDim.x * blockDim.x) >> 5;
-  for (int task = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; task < G.total_tasks; task += warps) {
-    int lo = 0, hi = G.count - 1;   // last problem with task_begin <= task
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (G.p[mid].task_begin <= task) lo = mid;
-      else hi = mid - 1;
-    }
-    const FwdProblem& P = G.p[lo];
-    const int row_blocks = P.n_out >> 4;
-    const int local = task - P.task_begin;
-    const int n0 = (local % row_blocks) * 16;
-    const int t0 = (local / row_blocks) * (8 * NG);
-    const int K = P.k_in;
-    const int kb = K >> 2;   // code bytes per row
-    const uint8_t* crow0 = P.codes + static_cast<int64_t>(n0 + g) * kb + tig * 16;
-    const uint8_t* crow1 = crow0 + 8 * static_cast<int64_t>(kb);
-    int acc[NG][4];
-#pragma unroll
-    for (int j = 0; j < NG; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0;
-    const int nchunks = (K + 255) >> 8;
-    const uint4 zero = make_uint4(0, 0, 0, 0);
-    uint4 c0n = (64 * tig < K) ? ld_stream_u4(crow0) : zero;
-    uint4 c1n = (64 * tig < K) ? ld_stream_u4(crow1) : zero;
-    for (int ch = 0; ch < nchunks; ++ch) {
-      const uint4 c0 = c0n, c1 = c1n;
-      const bool mine = ch * 256 + 64 * tig < K;   // this thread's 64 weights exist
-      if (ch + 1 < nchunks) {
-        const bool next = (ch + 1) * 256 + 64 * tig < K;
-        c0n = next ? ld_stream_u4(crow0 + (ch + 1) * 64) : zero;
-        c1n = next ? ld_stream_u4(crow1 + (ch + 1) * 64) : zero;
+  const int warps = gridDim.x * C::kWarps;
+  const int tok_per_task = 8 * NG;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+
+  // producer cursor: (task, chunk) running kDecDepth chunks ahead, across tasks
+  int p_task = blockIdx.x * C::kWarps + wid, p_ch = 0;
+  DecTask pd;
+  if (p_task < G.total_tasks) pd = dec_task(G, p_task, tok_per_task);
+  int issued = 0;
+  auto produce_one = [&]() {   // always commits one group (empty past the end)
+    if (p_task < G.total_tasks) {
+      const int kb = pd.P->k_in >> 2;
+      const bool valid = p_ch * 256 + 64 * tig < pd.P->k_in;
+      const uint8_t* src = pd.P->codes + static_cast<int64_t>(pd.n0 + g) * kb + p_ch * 64 + tig * 16;
+      const uint32_t dst = ring + static_cast<uint32_t>(issued % kDecDepth) * kSlot;
+      cp_async16(dst, valid ? src : pd.P->codes, valid);
+      cp_async16(dst + kHalf, valid ? src + 8 * static_cast<int64_t>(kb) : pd.P->codes, valid);
+      if (++p_ch == pd.nch) {
+        p_ch = 0;
+        p_task += warps;
+        if (p_task < G.total_tasks) pd = dec_task(G, p_task, tok_per_task);
       }
+    }
+    cp_async_commit();
+    ++issued;
+  };
+#pragma unroll
+  for (int i = 0; i < kDecDepth - 1; ++i) produce_one();
+
+  int consumed = 0;
+  for (int task = blockIdx.x * C::kWarps + wid; task < G.total_tasks; task += warps) {
+    const DecTask d = dec_task(G, task, tok_per_task);
+    const FwdProblem& P = *d.P;
+    const int K = P.k_in;
+    const int8_t* xrow[NG];
+#pragma unroll
+    for (int j = 0; j < NG; ++j) {
+      const int tok = min(d.t0 + 8 * j + g, P.t - 1);   // past-the-end tokens feed unstored columns
+      xrow[j] = P.xq + static_cast<int64_t>(tok) * K + tig * 64;
+    }
+    DecAcc<NG> accs;
+#pragma unroll
+    for (int k = 0; k < DecAcc<NG>::kSets; ++k)
+#pragma unroll
+      for (int j = 0; j < NG; ++j) accs.v[k][j][0] = accs.v[k][j][1] = accs.v[k][j][2] = accs.v[k][j][3] = 0;
+    for (int ch = 0; ch < d.nch; ++ch) {
+      produce_one();                      // chunk consumed + kDecDepth - 1
+      cp_async_wait<kDecDepth - 1>();     // chunk `consumed` has landed (own copies only)
+      const uint32_t slot = ring + static_cast<uint32_t>(consumed % kDecDepth) * kSlot;
+      uint4 c0, c1;
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(c0.x), "=r"(c0.y), "=r"(c0.z), "=r"(c0.w) : "r"(slot));
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w)
+                   : "r"(slot + kHalf));
+      ++consumed;
+      const bool mine = ch * 256 + 64 * tig < K;
       uint4 xv[NG][4];
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
-        const int tok = t0 + 8 * j + g;
-        const bool ok = mine && tok < P.t;
-        const uint4* xp = reinterpret_cast<const uint4*>(P.xq + static_cast<int64_t>(tok) * K + ch * 256 + tig * 64);
+        const uint4* xp = reinterpret_cast<const uint4*>(xrow[j] + ch * 256);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) xv[j][q] = ok ? __ldg(xp + q) : zero;
+        for (int q = 0; q < 4; ++q) xv[j][q] = mine ? __ldg(xp + q) : zero;
       }
-#pragma unroll
-      for (int st = 0; st < 8; ++st) {
-        const uint32_t a0 = my_lut[byte_of(c0, 2 * st) << 5];
-        const uint32_t a2 = my_lut[byte_of(c0, 2 * st + 1) << 5];
-        const uint32_t a1 = my_lut[byte_of(c1, 2 * st) << 5];
-        const uint32_t a3 = my_lut[byte_of(c1, 2 * st + 1) << 5];
-#pragma unroll
-        for (int j = 0; j < NG; ++j) {
-          const uint4& xa = xv[j][st >> 1];
-          const uint32_t b0 = (st & 1) ? xa.z : xa.x;
-          const uint32_t b1 = (st & 1) ? xa.w : xa.y;
-          mma_m16n8k32_s8(acc[j], a0, a1, a2, a3, b0, b1);
-        }
-      }
+      decode_chunk<NG>(accs, lut, lane4, c0, c1, xv);
     }
+    int acc[NG][4];
+#pragma unroll
+    for (int j = 0; j < NG; ++j)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        int sum = 0;
+#pragma unroll
+        for (int k = 0; k < DecAcc<NG>::kSets; ++k) sum += accs.v[k][j][v];
+        acc[j][v] = sum;
+      }
     // C fragment: acc[j][0..1] = row g, tokens 2*tig, 2*tig+1; acc[j][2..3] = row g+8
     const float gamma = *P.w_scale;
 #pragma unroll
     for (int j = 0; j < NG; ++j) {
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const int tok = t0 + 8 * j + 2 * tig + (v & 1);
-        const int n = n0 + g + ((v >> 1) << 3);
+        const int tok = d.t0 + 8 * j + 2 * tig + (v & 1);
+        const int n = d.n0 + g + ((v >> 1) << 3);
         if (tok < P.t) {
           const float rs = __fmul_rn(__fdiv_rn(P.absmax[tok], 127.0f), gamma);
           const float y = __fmul_rn(static_cast<float>(acc[j][v]), rs);
@@ -189,6 +304,7 @@ __global__ void __launch_bounds__(kDecodeThreads) fwd_codes_mma_kernel(const __g
       }
     }
   }
+  cp_async_wait<0>();   // no copy in flight when the thread exits
 }
 
 }  // namespace bl

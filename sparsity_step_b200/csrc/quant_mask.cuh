@@ -6,58 +6,63 @@
 // BitNet b1.58 2B4T article (lsdiaocha.cn), section 一: absmean quantisation to
 // {-1, 0, +1}; section 四: four ternary values packed per byte.
 //
-// Three launches, all HBM-bound:
-//   qm_abs_sum_kernel   : grid-stride read of W (16-byte vector loads), per-block
-//                         exact integer sum of floor(|w| * 2^32) -> workspace.
-//   qm_finalize_kernel  : one block; sums the block partials (128-bit), rounds
-//                         S / (n * 2^32) once to fp32, gamma = mean + 1e-5.
+// Two launches, both HBM-bound:
+//   qm_abs_sum_kernel   : grid-stride read of W (four 16-byte loads in flight per
+//                         thread), per-block exact integer sum of floor(|w| * 2^32);
+//                         the last block adds the partials (128-bit), rounds
+//                         S / (n * 2^32) once to fp32 and writes gamma = mean + 1e-5.
 //   qm_mask_codes_kernel: one thread per 8 contiguous weights (two 16-byte loads,
-//                         a warp covers 1 KB contiguous); rank-based top-N mask,
-//                         ternary codes, 2-bit packing, optional int8 weights.
+//                         a warp covers 1 KB contiguous); top-N mask by selection
+//                         scans, ternary codes, 2-bit packing, optional int8 weights.
 #pragma once
 
 #include "common.cuh"
 
 namespace bl {
 
-// Workspace layout (bytes): [0,4) range flag, [4,8) status, [8,16) reserved,
-// [256, 256 + 16 * blocks) per-block 128-bit partial sums (lo, hi).
+// Workspace layout (bytes): [0,4) range flag, [4,8) status, [8,12) blocks done,
+// [12,16) reserved, [256, 256 + 16 * blocks) per-block 128-bit partial sums (lo, hi).
+// The first 16 bytes must be zero when a call starts (the host clears them).
 constexpr size_t kQmWsHeader = 256;
 constexpr int kQmThreads = 256;
+constexpr int kQmUnroll = 4;                        // 16-byte loads in flight per thread
 constexpr int64_t kQmMaxElemsPerThread = 1 << 14;   // keeps a thread's u64 sum < 2^62
 constexpr float kAbsLimit = 65536.0f;              // |w| < 2^16 is summed exactly
 
-__global__ void __launch_bounds__(kQmThreads) qm_abs_sum_kernel(const float4* __restrict__ w4, int64_t n4,
-                                                                 unsigned long long* __restrict__ partials,
-                                                                 unsigned int* __restrict__ range_flag) {
-  uint64_t acc = 0;
-  bool bad = false;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
-    const float4 v = __ldcs(w4 + i);   // streamed: read once here
-    const float e[4] = {v.x, v.y, v.z, v.w};
+struct QmScratch {
+  unsigned int* range_flag;
+  int* status;
+  unsigned int* done;
+  unsigned long long* partials;
+};
+
+__device__ __forceinline__ void qm_accumulate(const float4& v, uint64_t& acc, bool& bad) {
+  const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float a = fabsf(e[j]);
-      if (a < kAbsLimit) {
-        // a * 2^32 is exact (power-of-two scale, < 2^48); truncation toward zero is floor
-        acc += __float2ull_rz(a * 4294967296.0f);
-      } else {
-        bad = true;   // also catches NaN (the comparison is false)
-      }
+  for (int j = 0; j < 4; ++j) {
+    const float a = fabsf(e[j]);
+    if (a < kAbsLimit) {
+      // a * 2^32 is exact (power-of-two scale, < 2^48); truncation toward zero is floor
+      acc += __float2ull_rz(a * 4294967296.0f);
+    } else {
+      bad = true;   // also catches NaN (the comparison is false)
     }
   }
-  if (bad) atomicOr(range_flag, 1u);
+}
 
-  uint64_t lo = acc, hi = 0;
+__device__ float rn_f32_ratio_u128(uint64_t slo, uint64_t shi, int64_t numel);
+
+// Block-reduce a 128-bit value held by every thread; the result is valid in thread 0.
+__device__ __forceinline__ void block_sum_u128(uint64_t& lo, uint64_t& hi) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     const uint64_t lo2 = __shfl_xor_sync(0xffffffffu, lo, off);
     const uint64_t hi2 = __shfl_xor_sync(0xffffffffu, hi, off);
     add_u128(lo, hi, lo2, hi2);
   }
-  __shared__ uint64_t s_lo[kQmThreads / 32], s_hi[kQmThreads / 32];
+  __shared__ uint64_t s_lo[32], s_hi[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();   // s_lo/s_hi may be reused by a previous call in this block
   if (lane == 0) {
     s_lo[warp] = lo;
     s_hi[warp] = hi;
@@ -65,10 +70,60 @@ __global__ void __launch_bounds__(kQmThreads) qm_abs_sum_kernel(const float4* __
   __syncthreads();
   if (threadIdx.x == 0) {
     uint64_t blo = 0, bhi = 0;
-    for (int w = 0; w < kQmThreads / 32; ++w) add_u128(blo, bhi, s_lo[w], s_hi[w]);
-    partials[2 * blockIdx.x] = blo;
-    partials[2 * blockIdx.x + 1] = bhi;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) add_u128(blo, bhi, s_lo[w], s_hi[w]);
+    lo = blo;
+    hi = bhi;
   }
+}
+
+// Pass 1: exact integer sum of floor(|w| * 2^32). Each block stores its partial; the
+// last block to finish (atomic ticket) adds all partials, rounds the mean once to
+// fp32, writes gamma = mean + 1e-5 (NaN and status BL_ERR_RANGE on a range error)
+// and clears the ticket and the flag for the next call.
+__global__ void __launch_bounds__(kQmThreads) qm_abs_sum_kernel(const float4* __restrict__ w4, int64_t n4, int64_t numel,
+                                                                 QmScratch ws, float* __restrict__ gamma_out) {
+  uint64_t acc = 0;
+  bool bad = false;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + (kQmUnroll - 1) * stride < n4; i += kQmUnroll * stride) {
+    float4 v[kQmUnroll];
+#pragma unroll
+    for (int u = 0; u < kQmUnroll; ++u) v[u] = __ldcs(w4 + i + u * stride);   // read once: streamed
+#pragma unroll
+    for (int u = 0; u < kQmUnroll; ++u) qm_accumulate(v[u], acc, bad);
+  }
+  for (; i < n4; i += stride) qm_accumulate(__ldcs(w4 + i), acc, bad);
+  if (bad) atomicOr(ws.range_flag, 1u);
+
+  uint64_t lo = acc, hi = 0;
+  block_sum_u128(lo, hi);
+  __shared__ bool s_last;
+  if (threadIdx.x == 0) {
+    ws.partials[2 * blockIdx.x] = lo;
+    ws.partials[2 * blockIdx.x + 1] = hi;
+    __threadfence();   // the partial is visible before the ticket is taken
+    s_last = atomicAdd(ws.done, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  lo = 0;
+  hi = 0;
+  for (int b = threadIdx.x; b < static_cast<int>(gridDim.x); b += blockDim.x)
+    add_u128(lo, hi, __ldcg(ws.partials + 2 * b), __ldcg(ws.partials + 2 * b + 1));
+  block_sum_u128(lo, hi);
+  if (threadIdx.x != 0) return;
+  const unsigned int flag = atomicAdd(ws.range_flag, 0u);
+  *ws.range_flag = 0;   // leave the scratch ready for the next call
+  *ws.done = 0;
+  if (flag) {
+    *ws.status = -4;   // BL_ERR_RANGE
+    *gamma_out = __int_as_float(0x7fc00000);
+    return;
+  }
+  *ws.status = 0;
+  *gamma_out = __fadd_rn(rn_f32_ratio_u128(lo, hi, numel), 1e-5f);   // one fp32 add
 }
 
 // ---- exact rounding of S / D to fp32 (round to nearest, ties to even) ----------
@@ -125,39 +180,68 @@ __device__ float rn_f32_ratio(U128 s, U128 d) {
   return ldexpf(static_cast<float>(m), e);   // exact: 24-bit mantissa, normal range
 }
 
-__global__ void qm_finalize_kernel(const unsigned long long* __restrict__ partials, int nblocks, int64_t numel,
-                                   unsigned int* __restrict__ range_flag, int* __restrict__ status,
-                                   float* __restrict__ gamma_out) {
-  uint64_t lo = 0, hi = 0;
-  for (int b = threadIdx.x; b < nblocks; b += blockDim.x) add_u128(lo, hi, partials[2 * b], partials[2 * b + 1]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const uint64_t lo2 = __shfl_xor_sync(0xffffffffu, lo, off);
-    const uint64_t hi2 = __shfl_xor_sync(0xffffffffu, hi, off);
-    add_u128(lo, hi, lo2, hi2);
-  }
-  __shared__ uint64_t s_lo[32], s_hi[32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) {
-    s_lo[warp] = lo;
-    s_hi[warp] = hi;
-  }
-  __syncthreads();
-  if (threadIdx.x != 0) return;
-  uint64_t slo = 0, shi = 0;
-  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) add_u128(slo, shi, s_lo[w], s_hi[w]);
-  const unsigned int bad = *range_flag;
-  *range_flag = 0;   // leave the workspace ready for the next call
-  if (bad) {
-    *status = -4;   // BL_ERR_RANGE
-    *gamma_out = __int_as_float(0x7fc00000);
-    return;
-  }
-  // mean = S / (numel * 2^32), rounded once; gamma = mean + 1e-5 (one fp32 add)
+// mean = S / (numel * 2^32), rounded once to fp32.
+__device__ float rn_f32_ratio_u128(uint64_t slo, uint64_t shi, int64_t numel) {
   const U128 den = shl_u128(U128{static_cast<uint64_t>(numel), 0}, 32);
-  const float mean = rn_f32_ratio(U128{slo, shi}, den);
-  *status = 0;
-  *gamma_out = __fadd_rn(mean, 1e-5f);
+  return rn_f32_ratio(U128{slo, shi}, den);
+}
+
+
+// Keep-mask of one group of M (weights [G0, G0+M) of the 8 held by the thread).
+// Element j outranks i when |w_j| > |w_i|, or they are equal and j < i (lower index
+// wins). NK > 0: compile-time N, found by selection scans: NK >= M/2 removes the
+// (M - NK) weakest one at a time, NK < M/2 picks the NK strongest; each scan is one
+// pass of compares in index order. NK == 0: runtime N via rank counting.
+template <int M, int NK, int G0>
+__device__ __forceinline__ uint32_t group_keep(const uint32_t (&a)[8], int n_keep) {
+  constexpr uint32_t all = (1u << M) - 1u;
+  if (NK == M) return all << G0;
+  if (NK > 0 && 2 * NK >= M) {
+    uint32_t dropped = 0;
+#pragma unroll
+    for (int r = 0; r < M - NK; ++r) {
+      uint32_t best_a = 0xFFFFFFFFu;
+      int best_j = 0;
+#pragma unroll
+      for (int j = 0; j < M; ++j) {
+        // scanning in index order, a later equal element is weaker: <= picks it
+        const bool take = !((dropped >> j) & 1u) && a[G0 + j] <= best_a;
+        best_a = take ? a[G0 + j] : best_a;
+        best_j = take ? j : best_j;
+      }
+      dropped |= 1u << best_j;
+    }
+    return (all & ~dropped) << G0;
+  }
+  if (NK > 0) {
+    uint32_t kept = 0;
+#pragma unroll
+    for (int r = 0; r < NK; ++r) {
+      int best_a = -1;
+      int best_j = 0;
+#pragma unroll
+      for (int j = 0; j < M; ++j) {
+        // scanning in index order, a later equal element is not stronger: strict >
+        const bool take = !((kept >> j) & 1u) && static_cast<int>(a[G0 + j]) > best_a;
+        best_a = take ? static_cast<int>(a[G0 + j]) : best_a;
+        best_j = take ? j : best_j;
+      }
+      kept |= 1u << best_j;
+    }
+    return kept << G0;
+  }
+  uint32_t keep = 0;
+#pragma unroll
+  for (int j = 0; j < M; ++j) {
+    int rank = 0;
+#pragma unroll
+    for (int t = 0; t < M; ++t) {
+      if (t == j) continue;
+      rank += (t < j) ? (a[G0 + t] >= a[G0 + j] ? 1 : 0) : (a[G0 + t] > a[G0 + j] ? 1 : 0);
+    }
+    keep |= (rank < n_keep ? 1u : 0u) << j;
+  }
+  return keep << G0;
 }
 
 // Ternary code of one weight. Equivalent, bit for bit, to
@@ -167,14 +251,11 @@ __global__ void qm_finalize_kernel(const unsigned long long* __restrict__ partia
 // the even 0.5), and no fp32 lies in (0.5 * gamma, 0.5 * gamma * (1 + 2^-24)] since
 // the spacing just above 0.5 * gamma is at least 0.5 * gamma * 2^-23 ... 2^-24 with
 // strict inequality (mantissa < 2^24). Quotients >= 1.5 round to 2 and clip to 1.
-// So code = sign(w) when |w| > 0.5 * gamma (0.5 * gamma exact in fp32), else 0.
-__device__ __forceinline__ int ternary_code(float w, float half_gamma) {
-  const float a = fabsf(w);
-  return (a > half_gamma) ? (w > 0.0f ? 1 : -1) : 0;
-}
-
+// So code = sign(w) when |w| > 0.5 * gamma (0.5 * gamma exact in fp32), else 0;
+// on the bit patterns of non-negative floats the comparison is an unsigned compare.
+//
 // One thread = 8 contiguous weights (one group of 8, or two groups of 4).
-template <int M>
+template <int M, int NK>
 __global__ void __launch_bounds__(kQmThreads) qm_mask_codes_kernel(const float4* __restrict__ w4, int64_t n8, int n_keep,
                                                                     const float* __restrict__ gamma_ptr,
                                                                     uint8_t* __restrict__ mask_out,
@@ -183,50 +264,35 @@ __global__ void __launch_bounds__(kQmThreads) qm_mask_codes_kernel(const float4*
   static_assert(M == 4 || M == 8, "groups of 4 or 8");
   const float gamma = *gamma_ptr;
   const bool gamma_ok = isfinite(gamma) && gamma > 0.0f;
-  const float half_gamma = 0.5f * gamma;   // exact
+  const uint32_t half_gamma_bits = __float_as_uint(0.5f * gamma);   // 0.5 * gamma is exact
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
     const float4 v0 = __ldcs(w4 + 2 * i);
     const float4 v1 = __ldcs(w4 + 2 * i + 1);
-    const float x[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const uint32_t b[8] = {__float_as_uint(v0.x), __float_as_uint(v0.y), __float_as_uint(v0.z), __float_as_uint(v0.w),
+                           __float_as_uint(v1.x), __float_as_uint(v1.y), __float_as_uint(v1.z), __float_as_uint(v1.w)};
     uint32_t a[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) a[j] = __float_as_uint(x[j]) & 0x7fffffffu;   // |w| bits: order-preserving
+    for (int j = 0; j < 8; ++j) a[j] = b[j] & 0x7fffffffu;   // |w| bits: order-preserving
+    uint32_t keep = group_keep<M, NK, 0>(a, n_keep);
+    if (M == 4) keep |= group_keep<M, NK, 4>(a, n_keep);
+    const uint32_t code_keep = gamma_ok ? keep : 0u;   // range error: all codes 0 (gamma is NaN)
 
-    // rank_j = #{i in group: |w_i| > |w_j| or (|w_i| == |w_j| and i < j)}; keep iff rank_j < N
-    uint32_t keep = 0;
+    uint32_t packed = 0, lo = 0, hi = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int g0 = (j / M) * M;
-      int rank = 0;
-#pragma unroll
-      for (int t = 0; t < M; ++t) {
-        const int ii = g0 + t;
-        if (ii == j) continue;
-        rank += (ii < j) ? (a[ii] >= a[j] ? 1 : 0) : (a[ii] > a[j] ? 1 : 0);
-      }
-      keep |= (rank < n_keep ? 1u : 0u) << j;
-    }
-
-    uint32_t packed = 0;
-    uint32_t lo = 0, hi = 0;   // int8 weights, little-endian
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      int c = gamma_ok ? ternary_code(x[j], half_gamma) : 0;
-      if (!((keep >> j) & 1u)) c = 0;
-      const uint32_t enc = (c == 0) ? 0u : (c > 0 ? 1u : 3u);   // 00 = 0, 01 = +1, 11 = -1
+      const uint32_t nz = ((code_keep >> j) & 1u) & (a[j] > half_gamma_bits ? 1u : 0u);
+      const uint32_t neg = b[j] >> 31;
+      const uint32_t enc = nz * (1u | (neg << 1));                 // 00 = 0, 01 = +1, 11 = -1
+      const uint32_t byte = nz * (neg ? 0xFFu : 0x01u);           // int8 -1 / +1 / 0
       packed |= enc << (2 * j);
-      const uint32_t byte = static_cast<uint32_t>(static_cast<uint8_t>(static_cast<int8_t>(c)));
       if (j < 4) lo |= byte << (8 * j);
       else hi |= byte << (8 * (j - 4));
     }
     codes_out[i] = static_cast<uint16_t>(packed);
     if (mask_out != nullptr) {
-      if (M == 8) {
-        mask_out[i] = static_cast<uint8_t>(keep);
-      } else {
-        reinterpret_cast<uint16_t*>(mask_out)[i] = static_cast<uint16_t>((keep & 0xFu) | ((keep >> 4) << 8));
-      }
+      if (M == 8) mask_out[i] = static_cast<uint8_t>(keep);
+      else reinterpret_cast<uint16_t*>(mask_out)[i] = static_cast<uint16_t>((keep & 0xFu) | ((keep >> 4) << 8));
     }
     if (w_i8_out != nullptr) w_i8_out[i] = make_uint2(lo, hi);
   }
