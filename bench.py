@@ -41,7 +41,11 @@ CFG_INDEX = 4   # the training-step workload's seed block
 # DRAM traffic per launch of the dominant kernel from an ncu capture, keyed by the
 # SHA-256 of the kernel's source files at capture time (reported as null once the
 # source has changed).
-TRAFFIC = {}
+TRAFFIC = {
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum (1 pass) on the full-size
+    # grad_W launch (16384 x 2048 x 11008): 701,756,416 B read + 41,950,208 B written
+    "bwd_grad_w": {"sha": "8b8bdb66281a51bd", "bytes": 743706624},
+}
 
 
 def kernel_source_sha() -> str:
@@ -727,6 +731,57 @@ def run_decode(args) -> None:
     print(json.dumps(res), flush=True)
 
 
+SWEEP_SHAPES = {
+    "qwen2.5-0.5b T=4096": (4096, [("q", 896, 896), ("k", 896, 128), ("v", 896, 128), ("o", 896, 896),
+                                   ("gate", 896, 4864), ("up", 896, 4864), ("down", 4864, 896)]),
+    "qwen2.5-1.5b-mlp T=8192": (8192, [("gate", 1536, 8960), ("up", 1536, 8960), ("down", 8960, 1536)]),
+}
+SWEEP_NM = [(8, 8), (6, 8), (4, 8), (2, 4), (2, 8)]
+
+
+def run_sweep(args) -> None:
+    """Forward product per shape (inference: masks and codes precomputed) for the
+    Qwen2.5-0.5B linears at 4096 tokens and the Qwen2.5-1.5B MLP at 8192 tokens,
+    for every N:M of the sweep: time, dense-equivalent and useful TOPS, and the
+    speedup over 8:8 of the same shape. Prints one JSON line."""
+    import numpy as np
+    import torch
+
+    import sparsity_step_b200 as B
+    from sparsity_step_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    res = {"workload": "forward per shape, N:M sweep", "shapes": {}}
+    for wl, (t, shapes) in SWEEP_SHAPES.items():
+        for name, k_in, n_out in shapes:
+            x = torch.from_numpy(synth.activation_bf16(synth.config_seed(3, 50 + k_in % 97), t, k_in).view(np.int16)).to(dev)
+            x = x.view(torch.bfloat16)
+            xq, a = B.bitlinear_act_quant(x)
+            w = torch.from_numpy(synth.latent_weight(synth.config_seed(3, 60 + n_out % 89), n_out, k_in)).to(dev)
+            y = torch.empty((t, n_out), dtype=torch.bfloat16, device=dev)
+            row = {}
+            for n, m in SWEEP_NM:
+                qm = B.bitlinear_quant_mask(w, n, m)
+                for _ in range(args.warmup):
+                    B.bitlinear_fwd(xq, a, qm["w_scale"], w_i8=qm["w_i8"], y=y)
+                torch.cuda.synchronize()
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record()
+                for _ in range(args.steps):
+                    B.bitlinear_fwd(xq, a, qm["w_scale"], w_i8=qm["w_i8"], y=y)
+                e.record()
+                torch.cuda.synchronize()
+                ms = s.elapsed_time(e) / args.steps
+                ops = 2.0 * t * k_in * n_out
+                row[f"{n}:{m}"] = {"us": round(ms * 1e3, 2), "tops_dense_equiv": round(ops / (ms * 1e-3) / 1e12, 1),
+                                   "tops_useful": round(ops * n / m / (ms * 1e-3) / 1e12, 1)}
+            base = row["8:8"]["us"]
+            for k in row:
+                row[k]["speedup_vs_8_8"] = round(base / row[k]["us"], 4)
+            res["shapes"][f"{wl} {name} {k_in}->{n_out}"] = row
+    print(json.dumps(res), flush=True)
+
+
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -744,7 +799,7 @@ def main(argv=None) -> None:
     ap.add_argument("--case-t", type=int, default=TOKENS)
     ap.add_argument("--case-k", type=int, default=2048)
     ap.add_argument("--case-n", type=int, default=11008)
-    ap.add_argument("--workload", choices=["train", "decode"], default="train",
+    ap.add_argument("--workload", choices=["train", "decode", "sweep"], default="train",
                     help="decode: the 36-layer stack at decode batches and prefill (separate JSON line)")
     ap.add_argument("--batches", type=int, nargs="+", default=[1, 8, 32, 128])
     ap.add_argument("--prefill", type=int, default=8192, help="prefill tokens for --workload decode (0 = skip)")
@@ -752,6 +807,9 @@ def main(argv=None) -> None:
     args = ap.parse_args(argv)
     if args.workload == "decode":
         run_decode(args)
+        return
+    if args.workload == "sweep":
+        run_sweep(args)
         return
     if args.case:
         run_case(args)
