@@ -134,6 +134,39 @@ def gpu_smi_id(local: int) -> str:
         return str(local)
 
 
+class RankSync:
+    """Barrier and max-over-ranks of the timed regions (the only collectives of the
+    benchmark; the data path has none). Works on any torch.distributed backend: on
+    NCCL the reduction tensor lives on this rank's GPU, on gloo on the CPU."""
+
+    def __init__(self, world: int, device=None):
+        self.world = world
+        self.device = device
+
+    def barrier(self) -> None:
+        if self.world > 1:
+            import torch.distributed as dist
+            if self.device is not None and self.device.type == "cuda":
+                dist.barrier(device_ids=[self.device.index])
+            else:
+                dist.barrier()
+
+    def max(self, v: float) -> float:
+        if self.world == 1:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=self.device if self.device is not None else "cpu")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def job_tokens_per_s(ms_per_step: float, world: int) -> float:
+    """Whole-job throughput: every rank processes its own TOKENS per step (weak
+    scaling); the step time is the max over ranks."""
+    return TOKENS * world / (ms_per_step * 1e-3)
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def make_inputs(rank: int):
@@ -323,16 +356,9 @@ def run_ours(args) -> None:
     step = Step(host, dev, n_io=2)
     stream = torch.cuda.current_stream()
 
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local])
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    sync = RankSync(world, dev)
+    barrier = sync.barrier
+    max_over_ranks = sync.max
 
     for _ in range(args.warmup):
         step.run()
@@ -408,7 +434,7 @@ def run_ours(args) -> None:
     else:
         roof = {"kernel": dominant, "bound": "unknown"}
 
-    tok_s = TOKENS * world / (ms_step * 1e-3)
+    tok_s = job_tokens_per_s(ms_step, world)
     out = {
         "metric": METRIC,
         "value": round(tok_s, 1),
@@ -434,7 +460,7 @@ def run_ours(args) -> None:
         "speedup_vs_8_8": round(ms_dense / ms_step, 4),
         "ms_per_step_8_8": round(ms_dense, 4),
         "roofline": roof,
-        "e2e": {"value": round(TOKENS * world / (ms_e2e * 1e-3), 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": round(job_tokens_per_s(ms_e2e, world), 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 3), "steps": e2e_steps,
                 "copies": "pinned host <-> device on separate H2D / D2H streams, overlapped with compute (2 I/O sets)"},
         "gpu_launches": step.launches_per_step * args.steps,
@@ -459,25 +485,37 @@ def _blas_threads() -> int:
         return 1
 
 
-def oracle_sample(tokens: int, w_rows: int | None, seed_off: int = 0) -> dict:
-    """Time the oracle on a bounded sample: the mask/code recompute of the three
-    weight tensors (all rows, or the first ``w_rows``), and ``tokens`` tokens through
-    act-quant, forward and both gradients. Returns the seconds of each part."""
-    from oracle import bitlinear_oracle as O
+def oracle_inputs(tokens: int, w_rows: int | None, seed_off: int = 0) -> list:
+    """Seeded inputs of a bounded oracle sample: per linear, the first ``w_rows`` rows
+    of the latent weights (all rows when None) and ``tokens`` tokens of X and dY."""
     from sparsity_step_b200 import synth
 
-    t_mask = 0.0
-    t_tok = 0.0
+    out = []
     for i, (name, k_in, n_out) in enumerate(LINEARS):
         rows = n_out if w_rows is None else min(w_rows, n_out)
         w = synth.latent_weight(synth.config_seed(CFG_INDEX, 3 * i) + seed_off, rows, k_in)
         x = synth.activation_bf16(synth.config_seed(CFG_INDEX, 3 * i + 1) + seed_off, tokens, k_in)
         dy = synth.activation_bf16(synth.config_seed(CFG_INDEX, 3 * i + 2) + seed_off, tokens, n_out, std=1e-2,
                                    outliers=False)
+        out.append((n_out, w, x, dy))
+    return out
+
+
+def oracle_sample(inputs: list) -> dict:
+    """Time the oracle on a bounded sample (see oracle_inputs): the mask/code recompute
+    of the sampled weight rows, scaled to all rows, and the sampled tokens through
+    act-quant, forward and both gradients against full-size code matrices, scaled to
+    the step's 16384 tokens. Returns the seconds of each part."""
+    from oracle import bitlinear_oracle as O
+
+    t_mask = 0.0
+    t_tok = 0.0
+    tokens = inputs[0][2].shape[0]
+    for n_out, w, x, dy in inputs:
+        rows = w.shape[0]
         s = time.perf_counter()
         qm = O.quant_mask(w, N_KEEP, M_GROUP)
         t_mask += (time.perf_counter() - s) * (n_out / rows)
-        # the token part runs against a full-size code matrix
         mcode = qm["mcode"] if rows == n_out else _tile_rows(qm["mcode"], n_out)
         s = time.perf_counter()
         q, a = O.act_quant(x)
@@ -496,7 +534,7 @@ def _tile_rows(a, n):
 
 
 def cpu_baseline(tokens: int) -> dict:
-    r = oracle_sample(tokens, None)
+    r = oracle_sample(oracle_inputs(tokens, None))
     return {"value": round(TOKENS / r["step_s"], 2), "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
             "sample": (f"full mask/ternary recompute of the 3 weight tensors ({r['mask_s']:.2f} s) + {tokens} of "
                        f"{TOKENS} tokens through act-quant/fwd/grad_x/grad_w ({r['tokens_s']:.2f} s), "
@@ -509,11 +547,12 @@ def run_reference(args) -> None:
     if rank != 0:
         return
     tokens, w_rows = args.ref_tokens, args.ref_w_rows
+    inputs = oracle_inputs(tokens, w_rows)
     for _ in range(args.warmup):
-        oracle_sample(tokens, w_rows)
+        oracle_sample(inputs)
     step_s = []
     for _ in range(args.steps):
-        step_s.append(oracle_sample(tokens, w_rows)["step_s"])
+        step_s.append(oracle_sample(inputs)["step_s"])
     ms = 1e3 * statistics.mean(step_s)
     v = round(TOKENS / (ms * 1e-3), 3)
     out = {
@@ -791,8 +830,8 @@ def main(argv=None) -> None:
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-tokens", type=int, default=256, help="tokens in the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-tokens", type=int, default=16, help="reference arm: tokens per sampled step")
-    ap.add_argument("--ref-w-rows", type=int, default=256, help="reference arm: weight rows per sampled step")
+    ap.add_argument("--ref-tokens", type=int, default=32, help="reference arm: tokens per sampled step")
+    ap.add_argument("--ref-w-rows", type=int, default=64, help="reference arm: weight rows per sampled step")
     ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_codes", "grad_x", "grad_w", "mma_peak_i8",
                              "mma_peak_bf16"],
                     help="time one kernel class alone on the --case-t/k/n shape")
