@@ -600,6 +600,32 @@ def mma_peak(kind: str, iters: int = 4000, reps: int = 3) -> float:
     return best
 
 
+def warp_mma_rate(kind: str, iters: int = 2000) -> dict:
+    """Rate of the legacy warp-level MMAs (mma.sync) from the probe library."""
+    import ctypes
+
+    import torch
+
+    lib = ctypes.CDLL(os.path.join(ROOT, "sparsity_step_b200", "libblprobe.so"))
+    lib.blprobe_warp_mma.restype = ctypes.c_int
+    lib.blprobe_warp_mma.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    k = 2 if kind == "s8" else 3
+    blocks = torch.cuda.get_device_properties(0).multi_processor_count * 4
+    st = torch.cuda.current_stream()
+    lib.blprobe_warp_mma(k, blocks, 10, st.cuda_stream)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(st)
+    if lib.blprobe_warp_mma(k, blocks, iters, st.cuda_stream) != 0:
+        raise RuntimeError("warp mma probe failed")
+    e.record(st)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    n_mma = blocks * 8 * iters * 8   # warps x iterations x MMAs
+    macs = 16 * 8 * (32 if kind == "s8" else 256)
+    return {"mma_per_s": n_mma / (ms * 1e-3), "ops_per_s": 2.0 * n_mma * macs / (ms * 1e-3),
+            "mma_per_sm_per_clk_at_1.9GHz": n_mma / (ms * 1e-3) / torch.cuda.get_device_properties(0).multi_processor_count / 1.9e9}
+
+
 def run_case(args) -> None:
     """One kernel class alone on a chosen shape (for ncu captures and tuning):
     warm-up launches, then ``--steps`` timed launches; prints one JSON line."""
@@ -609,6 +635,10 @@ def run_case(args) -> None:
     import sparsity_step_b200 as B
     from sparsity_step_b200 import synth
 
+    if args.case.startswith("warp_mma"):
+        kind = args.case.split("_")[-1]
+        print(json.dumps({"case": args.case, **warp_mma_rate(kind)}), flush=True)
+        return
     if args.case.startswith("mma_peak"):
         kind = args.case.split("_")[-1]
         print(json.dumps({"case": args.case, "rate": round(mma_peak(kind), 1),
@@ -833,7 +863,7 @@ def main(argv=None) -> None:
     ap.add_argument("--ref-tokens", type=int, default=32, help="reference arm: tokens per sampled step")
     ap.add_argument("--ref-w-rows", type=int, default=64, help="reference arm: weight rows per sampled step")
     ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_codes", "grad_x", "grad_w", "mma_peak_i8",
-                             "mma_peak_bf16"],
+                             "mma_peak_bf16", "warp_mma_s8", "warp_mma_b1"],
                     help="time one kernel class alone on the --case-t/k/n shape")
     ap.add_argument("--case-t", type=int, default=TOKENS)
     ap.add_argument("--case-k", type=int, default=2048)
