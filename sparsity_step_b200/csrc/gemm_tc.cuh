@@ -13,8 +13,9 @@
 //
 // Tile 128 x 256, K step 128 bytes (64 bf16 or 128 int8) per pipeline stage, 4
 // stages of 48 KB. Warp 0: TMA producer (one thread). Warp 1: TMEM allocator and
-// MMA issuer (one thread). Warps 2-5: epilogue (TMEM -> registers -> global), each
-// warp owning the 32 TMEM lanes (= tile rows) its warp-rank-in-quad may access.
+// MMA issuer (one thread). Warps 2-9: epilogue (TMEM -> registers -> global), two
+// warps on the 32 TMEM lanes (= tile rows) their warp-rank-in-quad may access, each
+// converting half of the tile's columns.
 // Two 256-column fp32/int32 accumulators in TMEM (all 512 columns) let the
 // epilogue of tile i overlap the main loop of tile i+1. Operands are staged with
 // 128-byte swizzle: K-major tiles are one TMA box of [rows x 128 B]; MN-major
@@ -34,12 +35,13 @@ constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBKBytes;   // 16 KB
 constexpr int kBBytes = kBN * kBKBytes;   // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter, half the columns each
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBarrierBytes = 256;
-// epilogue staging for TMA stores: per epilogue warp two buffers of 32 rows x 128 B
+// epilogue staging for TMA stores: per epilogue warp one buffer of 32 rows x 128 B
 constexpr int kStageOutBytes = 32 * 128;
-constexpr int kOutStagingBytes = 4 * 2 * kStageOutBytes;   // 32 KB
+constexpr int kOutStagingBytes = kEpiWarps * kStageOutBytes;   // 32 KB
 constexpr size_t gemm_smem_bytes(bool tma_store) {
   return 1024 + static_cast<size_t>(kStages) * kStageBytes + (tma_store ? kOutStagingBytes : 0) + kBarrierBytes;
 }
@@ -114,12 +116,12 @@ __device__ __forceinline__ void epilogue_store32(const GemmArgs& g, const uint32
 // and the layout the store's tensor map expects), then one lane stores the box.
 template <int kEpi>
 __device__ __forceinline__ void epilogue_tile_tma(const GemmArgs& g, const CUtensorMap* tmOut, uint32_t t_row,
-                                                  uint32_t stage_base, int& cnt, int row0, int n0, float rs, int lane) {
+                                                  uint32_t buf, int& cnt, int row0, int n0, int col_begin, float rs,
+                                                  int lane) {
   const int ecols = g.out_f32 ? 32 : 64;
-  for (int c = 0; c < kBN / ecols; ++c, ++cnt) {
-    const uint32_t buf = stage_base + static_cast<uint32_t>(cnt & 1) * kStageOutBytes;
-    if (cnt >= 2) {
-      if (lane == 0) bulk_wait_group_read<1>();   // the store that last read this buffer is done reading
+  for (int c = col_begin / ecols; c < (col_begin + kBN / 2) / ecols; ++c, ++cnt) {
+    if (cnt >= 1) {
+      if (lane == 0) bulk_wait_group_read<0>();   // the previous store has finished reading the buffer
       __syncwarp();
     }
     uint32_t r0[32], r1[32];
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8u * b, 1);
-      mbar_init(tempty0 + 8u * b, 4);   // one arrival per epilogue warp
+      mbar_init(tempty0 + 8u * b, kEpiWarps);   // one arrival per epilogue warp
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -319,24 +321,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!mbar_wait_plain(done_bar, 0)) atomicOr(&g_device_status, DEV_ST_TIMEOUT_DRAIN);
     }
   } else {
-    // ------------------------------------------------------------- epilogue (warps 2..5)
+    // ------------------------------------------------------------- epilogue (warps 2..9)
+    // two warps per TMEM lane quarter: warp 2+e owns lanes [32*quad, +32) and the
+    // column half e / 4 of each 256-column accumulator
+    const int e = warp - 2;
     const int quad = warp & 3;   // TMEM lanes [32*quad, 32*quad+32) belong to this warp
+    const int col_begin = (e >> 2) * (kBN / 2);
     const int row_in_tile = quad * 32 + lane;
     const float gamma = (kEpi == EPI_GRADW) ? 1.0f : *g.w_scale;
-    const uint32_t stage_base = sOut + static_cast<uint32_t>((warp - 2) * 2 * kStageOutBytes);
-    int cnt = 0;   // staging buffers used so far (double-buffered)
+    const uint32_t stage_buf = sOut + static_cast<uint32_t>(e * kStageOutBytes);
+    int cnt = 0;   // stores issued from the staging buffer so far
     int local = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int buf = local & 1;
       const uint32_t tph = static_cast<uint32_t>(local >> 1) & 1u;
-      // warp-uniform decision: the TMEM loads below are warp-collective
-      const bool got = mbar_wait(tfull0 + 8u * buf, tph, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after_sync();
+      // the row scale does not depend on the accumulator: fetch it before waiting
       const int row = (tile / g.num_n_blocks) * kBM + row_in_tile;
       const int n0 = (tile % g.num_n_blocks) * kBN;
       const bool row_ok = row < g.M;
@@ -346,12 +346,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       } else if (kEpi == EPI_GRADX) {
         rs = gamma;
       }
+      // warp-uniform decision: the TMEM loads below are warp-collective
+      const bool got = mbar_wait(tfull0 + 8u * buf, tph, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
       const uint32_t t_row = tmem_base + static_cast<uint32_t>(buf * kBN) + (static_cast<uint32_t>(quad * 32) << 16);
       if (kTmaStore) {
-        epilogue_tile_tma<kEpi>(g, &tmOut, t_row, stage_base, cnt, row - lane, n0, rs, lane);
+        epilogue_tile_tma<kEpi>(g, &tmOut, t_row, stage_buf, cnt, row - lane, n0, col_begin, rs, lane);
       } else {
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = col_begin / 32; c < (col_begin + kBN / 2) / 32; ++c) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * 32), r);
           tmem_ld_wait();
