@@ -11,6 +11,7 @@
 #include "codes_kernels.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "quant_mask.cuh"
 
 namespace {
@@ -107,6 +108,50 @@ bl_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return BL_OK;
 }
+
+// Two-SM version: clusters of two CTAs, each pair computing 256 x 256 output tiles
+// (g.num_m_blocks / g.num_n_blocks count 256-wide blocks). Sets *launched to false and
+// launches nothing when no CTA pair fits on the device, so the caller can fall back.
+template <bool kI8, bool kAMN, bool kBMN, int kEpi>
+bl_status launch_gemm2(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout, const bl::GemmArgs& g,
+                       cudaStream_t st, bool* launched) {
+  *launched = false;
+  auto kern = bl::gemm_tc2_kernel<kI8, kAMN, kBMN, kEpi>;
+  constexpr size_t smem = bl::gemm2_smem_bytes();
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(bl::kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters = -1;   // per instantiation
+  if (max_clusters < 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm2)");
+    cfg.gridDim = dim3(2 * (device_sm_count() / 2));
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(gemm2)");
+    max_clusters = n;
+  }
+  if (max_clusters <= 0) return BL_OK;
+  const int tiles = g.num_m_blocks * g.num_n_blocks;
+  const int clusters = tiles < max_clusters ? tiles : max_clusters;
+  cfg.gridDim = dim3(2 * clusters);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tout, g);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm2 launch");
+  *launched = true;
+  return BL_OK;
+}
+
+// Pairs pay off once the output has at least two 128-row blocks; a single block would
+// leave half of each pair's tensor work on rows outside the output.
+inline bool use_cta_pair(int64_t m) { return m > bl::kBM; }
 
 // ------------------------------------------------------------------ grouped codes product
 
@@ -340,6 +385,15 @@ bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* co
     }
     CUtensorMap to;
     if (bl_status s = make_out_map(&to, y_out, t, n_out, g.out_f32)) return s;
+    if (use_cta_pair(t)) {   // each CTA of a pair loads 128 of the tile's 256 weight rows
+      CUtensorMap tb2;
+      if (bl_status s = make_map(&tb2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_i8, k_in, n_out, 128, 128)) return s;
+      bl::GemmArgs g2 = g;
+      g2.num_m_blocks = static_cast<int>((t + 255) / 256);
+      bool launched = false;
+      if (bl_status s = launch_gemm2<true, false, false, bl::EPI_FWD>(ta, tb2, to, g2, st, &launched)) return s;
+      if (launched) return BL_OK;
+    }
     return launch_gemm<true, false, false, bl::EPI_FWD, true>(ta, tb, to, g, st);
   }
   bl_fwd_problem prob{xq, absmax, codes, w_scale, t, k_in, n_out, acc_out, y_out};
@@ -420,7 +474,14 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* co
     g.w_scale = w_scale;
     CUtensorMap to;
     if (bl_status s = make_out_map(&to, grad_x, t, k_in, false)) return s;
-    if (bl_status s = launch_gemm<false, false, true, bl::EPI_GRADX, true>(ta, tb, to, g, st)) return s;
+    bool launched = false;
+    if (use_cta_pair(t)) {
+      bl::GemmArgs g2 = g;
+      g2.num_m_blocks = static_cast<int>((t + 255) / 256);
+      if (bl_status s = launch_gemm2<false, false, true, bl::EPI_GRADX>(ta, tb, to, g2, st, &launched)) return s;
+    }
+    if (!launched)
+      if (bl_status s = launch_gemm<false, false, true, bl::EPI_GRADX, true>(ta, tb, to, g, st)) return s;
   }
   if (grad_w) {
     CUtensorMap ta, tb;
@@ -437,7 +498,14 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* co
     g.out_f32 = grad_w_dtype == BL_OUT_F32;
     CUtensorMap to;
     if (bl_status s = make_out_map(&to, grad_w, n_out, k_in, g.out_f32)) return s;
-    if (bl_status s = launch_gemm<false, true, true, bl::EPI_GRADW, true>(ta, tb, to, g, st)) return s;
+    bool launched = false;
+    if (use_cta_pair(n_out)) {
+      bl::GemmArgs g2 = g;
+      g2.num_m_blocks = static_cast<int>((n_out + 255) / 256);
+      if (bl_status s = launch_gemm2<false, true, true, bl::EPI_GRADW>(ta, tb, to, g2, st, &launched)) return s;
+    }
+    if (!launched)
+      if (bl_status s = launch_gemm<false, true, true, bl::EPI_GRADW, true>(ta, tb, to, g, st)) return s;
   }
   return BL_OK;
 }

@@ -204,6 +204,14 @@ def test_ragged_token_counts(t):
     full_layer(1, 10 + t, t, 576, 144, 6, 8)
 
 
+@pytest.mark.parametrize("t,n_out", [(128, 128), (129, 128), (128, 144), (257, 400), (520, 272)])
+def test_cta_pair_threshold(t, n_out):
+    # Products with more than 128 output rows run on CTA pairs (256-row tiles split
+    # over two SMs), the others on single CTAs: both sides of the switch, with rows
+    # of the last pair tile beyond the output and a ragged K (k_in = 320).
+    full_layer(1, 40 + t + n_out, t, 320, n_out, 6, 8)
+
+
 @pytest.mark.parametrize("nm", [(6, 8), (4, 8), (3, 8), (2, 4), (1, 4), (8, 8)])
 def test_mask_ties(nm):
     n, m = nm
