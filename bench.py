@@ -43,14 +43,15 @@ CFG_INDEX = 4   # the training-step workload's seed block
 # source has changed).
 TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum (1 pass) on the full-size
-    # grad_W launch (16384 x 2048 x 11008): 701,756,416 B read + 41,950,208 B written
-    "bwd_grad_w": {"sha": "8b8bdb66281a51bd", "bytes": 743706624},
+    # grad_W launch (16384 x 2048 x 11008, CTA-pair kernel): 722,842,368 B read +
+    # 41,942,272 B written
+    "bwd_grad_w": {"sha": "e3829fad9d296712", "bytes": 764784640},
 }
 
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("gemm_tc.cuh", "common.cuh"):
+    for f in ("gemm_tc.cuh", "gemm_tc2.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "sparsity_step_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -236,7 +237,9 @@ class Step:
         self.gw = {n: torch.empty((n_out, k_in), dtype=bf, device=dev) for n, k_in, n_out in LINEARS}
         wsb = max(B.bitlinear_bwd_workspace_size(T, k, n, True) for _, k, n in LINEARS)
         self.ws_bwd = torch.empty((wsb,), dtype=torch.uint8, device=dev)
-        self.launches_per_step = 3 * 3 + 2 + 3 + 3 * 3
+        # kernels per step: quant_mask 2 (plus a 16-byte memset, not a kernel), act_quant 1,
+        # fwd 1, grad_X 2 (expand + GEMM), grad_W 1
+        self.launches_per_step = 3 * 2 + 2 + 3 + 3 * 2 + 3
 
     def run(self, ev=None, io=0):
         """Enqueue one step on the current stream using I/O set ``io``. ``ev`` maps a
