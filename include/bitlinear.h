@@ -185,9 +185,11 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* co
                         int64_t k_in, int64_t n_out, uint16_t* grad_x, void* grad_w, int grad_w_dtype,
                         void* workspace, size_t workspace_bytes, void* stream);
 
-/* Synchronises the current device, then returns BL_OK, or BL_ERR_TIMEOUT if a
- * kernel of this library gave up on a bounded wait since the last call (the raw
- * status bits go to *bits when bits != NULL). Clears the status. */
+/* Synchronises the current device, then returns BL_OK; BL_ERR_TIMEOUT if a kernel
+ * of this library gave up on a bounded wait since the last call (bits 0-3); or
+ * BL_ERR_CUDA if the decode kernel found its dynamic shared memory at an address
+ * where its fixed-address lookup table does not fit and skipped its work (bit 4).
+ * The raw status bits go to *bits when bits != NULL. Clears the status. */
 bl_status bitlinear_device_status(unsigned int* bits);
 
 /* Message for the calling thread's last non-OK status ("" if none). */

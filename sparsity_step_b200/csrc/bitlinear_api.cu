@@ -520,6 +520,8 @@ bl_status bitlinear_device_status(unsigned int* bits) {
   e = cudaMemcpyToSymbol(bl::g_device_status, &zero, sizeof(zero));
   if (e != cudaSuccess) return cuda_fail(e, "status clear");
   if (bits) *bits = v;
+  if (v & bl::DEV_ST_SMEM_LAYOUT)
+    return fail(BL_ERR_CUDA, "a kernel found its shared memory at an unexpected address and skipped its work (status bits 0x%x)", v);
   if (v) return fail(BL_ERR_TIMEOUT, "a kernel gave up on a bounded wait (status bits 0x%x)", v);
   return BL_OK;
 }

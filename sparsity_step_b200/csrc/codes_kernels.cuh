@@ -92,13 +92,22 @@ __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
   return v;
 }
 
-// Table lookup of code byte j (0..3) of word w for this lane: entry e of lane l is the
-// 32-bit word at byte offset 128*e + 4*l of the table, so the offset is
-// ((w >> (8j - 7)) & 0x7F80) | 4*lane: one shift and one logic op, conflict-free.
+// The byte -> int8x4 table lives at a fixed shared-window address: entry e of lane l is
+// the word at kDecLutAddr + 256*e + 4*l (lanes use the first 128 bytes of each 256-byte
+// row), so each lane reads its own bank and the address of code byte j of word w is one
+// byte permute: byte 0 <- 4*lane, byte 1 <- byte j of w, byte 2 <- 0x01 (kDecLutAddr
+// >> 16), byte 3 <- 0. `lanesel` = 0x00010000 | 4*lane supplies bytes 0, 2 and 3.
+constexpr uint32_t kDecLutAddr = 0x10000;
+constexpr uint32_t kDecLutSpan = 256 * 256;
+constexpr uint32_t kDecHighBase = kDecLutAddr + kDecLutSpan;
+static_assert(kDecLutAddr == 0x10000, "lut_lookup builds byte 2 of the address from lanesel");
+
 template <int J>
-__device__ __forceinline__ uint32_t lut_lookup(const uint32_t* lut, uint32_t w, uint32_t lane4) {
-  const uint32_t off = ((J == 0 ? (w << 7) : (w >> (8 * J - 7))) & 0x7F80u) | lane4;
-  return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(lut) + off);
+__device__ __forceinline__ uint32_t lut_lookup(uint32_t w, uint32_t lanesel) {
+  const uint32_t addr = __byte_perm(w, lanesel, 0x7604u | (J << 4));
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
 // Accumulators per token group, optionally split into independent sets (summed at
@@ -112,48 +121,51 @@ struct DecAcc {
 
 // Two MMA steps from one 32-bit word of each row's codes (bytes 0..3 = steps 2h, 2h+1).
 template <int NG>
-__device__ __forceinline__ void decode_mma_word(DecAcc<NG>& acc, const uint32_t* lut, uint32_t lane4, uint32_t w0,
-                                                uint32_t w1, const uint4 (&xv)[NG][4], int h) {
+__device__ __forceinline__ void decode_mma_word(DecAcc<NG>& acc, uint32_t lanesel, uint32_t w0, uint32_t w1,
+                                                const uint4 (&xv)[NG][4], int h) {
   constexpr int S = DecAcc<NG>::kSets;
   {   // step 2h: bytes 0 (a0) and 1 (a2) of row g's word, of row g+8's word (a1, a3)
-    const uint32_t a0 = lut_lookup<0>(lut, w0, lane4), a2 = lut_lookup<1>(lut, w0, lane4);
-    const uint32_t a1 = lut_lookup<0>(lut, w1, lane4), a3 = lut_lookup<1>(lut, w1, lane4);
+    const uint32_t a0 = lut_lookup<0>(w0, lanesel), a2 = lut_lookup<1>(w0, lanesel);
+    const uint32_t a1 = lut_lookup<0>(w1, lanesel), a3 = lut_lookup<1>(w1, lanesel);
 #pragma unroll
     for (int j = 0; j < NG; ++j) mma_m16n8k32_s8(acc.v[(2 * h) % S][j], a0, a1, a2, a3, xv[j][h].x, xv[j][h].y);
   }
   {   // step 2h+1: bytes 2, 3
-    const uint32_t a0 = lut_lookup<2>(lut, w0, lane4), a2 = lut_lookup<3>(lut, w0, lane4);
-    const uint32_t a1 = lut_lookup<2>(lut, w1, lane4), a3 = lut_lookup<3>(lut, w1, lane4);
+    const uint32_t a0 = lut_lookup<2>(w0, lanesel), a2 = lut_lookup<3>(w0, lanesel);
+    const uint32_t a1 = lut_lookup<2>(w1, lanesel), a3 = lut_lookup<3>(w1, lanesel);
 #pragma unroll
     for (int j = 0; j < NG; ++j) mma_m16n8k32_s8(acc.v[(2 * h + 1) % S][j], a0, a1, a2, a3, xv[j][h].z, xv[j][h].w);
   }
 }
 
 template <int NG>
-__device__ __forceinline__ void decode_chunk(DecAcc<NG>& acc, const uint32_t* lut, uint32_t lane4, const uint4& c0,
-                                             const uint4& c1, const uint4 (&xv)[NG][4]) {
-  decode_mma_word<NG>(acc, lut, lane4, c0.x, c1.x, xv, 0);
-  decode_mma_word<NG>(acc, lut, lane4, c0.y, c1.y, xv, 1);
-  decode_mma_word<NG>(acc, lut, lane4, c0.z, c1.z, xv, 2);
-  decode_mma_word<NG>(acc, lut, lane4, c0.w, c1.w, xv, 3);
+__device__ __forceinline__ void decode_chunk(DecAcc<NG>& acc, uint32_t lanesel, const uint4& c0, const uint4& c1,
+                                             const uint4 (&xv)[NG][4]) {
+  decode_mma_word<NG>(acc, lanesel, c0.x, c1.x, xv, 0);
+  decode_mma_word<NG>(acc, lanesel, c0.y, c1.y, xv, 1);
+  decode_mma_word<NG>(acc, lanesel, c0.z, c1.z, xv, 2);
+  decode_mma_word<NG>(acc, lanesel, c0.w, c1.w, xv, 3);
 }
 
 // Per-thread streaming: each thread copies the 32 code bytes it will itself decode
 // per chunk (16 bytes of row g, 16 of row g+8) with cp.async into its own slots of a
 // shared-memory ring kDecDepth chunks deep, so up to kDecDepth chunks per warp are in
 // flight without holding registers, and no thread ever reads another thread's data.
-// Ring layout [chunk slot][row half][thread][16 B]: consecutive threads read
-// consecutive 16-byte slots (conflict-free).
+// Slot layout [row half][thread][16 B]: consecutive threads read consecutive 16-byte
+// slots (conflict-free). Slot 0 sits at the start of the dynamic shared memory, below
+// the table; slots 1.. sit above it, from kDecHighBase.
 constexpr int kDecDepth = 4;
-constexpr int kDecLutBytes = 256 * 32 * 4;
 
 template <int NG>
 struct DecCfg {
   static constexpr int kWarps = NG == 1 ? 32 : 16;
   static constexpr int kThreads = kWarps * 32;
-  static constexpr int kRingBytes = kDecDepth * 2 * kThreads * 16;
-  static constexpr int kSmemBytes = kDecLutBytes + kRingBytes;
+  static constexpr uint32_t kSlotBytes = 2u * kThreads * 16u;
+  // enough for any start address of the dynamic shared memory: the last slot ends at
+  // kDecHighBase + (kDecDepth - 1) * kSlotBytes
+  static constexpr int kSmemBytes = static_cast<int>(kDecHighBase + (kDecDepth - 1) * kSlotBytes);
 };
+static_assert(DecCfg<1>::kSmemBytes <= 232448, "decode ring and table exceed the shared memory of a CTA");
 
 struct DecTask {
   const FwdProblem* P;
@@ -192,46 +204,62 @@ template <int NG>   // token groups of 8 per task (1, 2 or 4)
 __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(const __grid_constant__ FwdGroup G) {
   using C = DecCfg<NG>;
   extern __shared__ __align__(1024) uint8_t dsmem[];
-  uint32_t* lut = reinterpret_cast<uint32_t*>(dsmem);
+  const uint32_t base = smem_u32(dsmem);
+  if (base + C::kSlotBytes > kDecLutAddr) {   // slot 0 would overlap the table: do nothing
+    if (threadIdx.x == 0) atomicOr(&g_device_status, DEV_ST_SMEM_LAYOUT);
+    return;
+  }
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-    const uint32_t e = static_cast<uint32_t>(i) >> 5;
+    const uint32_t e = static_cast<uint32_t>(i) >> 5, l = static_cast<uint32_t>(i) & 31u;
     uint32_t word = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t f = (e >> (2 * j)) & 3u;
       word |= ((f & 1u) ? ((f & 2u) ? 0xFFu : 0x01u) : 0u) << (8 * j);
     }
-    lut[i] = word;
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(kDecLutAddr + 256u * e + 4u * l), "r"(word) : "memory");
   }
   __syncthreads();
-  const uint32_t ring = smem_u32(dsmem + kDecLutBytes) + static_cast<uint32_t>(threadIdx.x * 16);
-  constexpr uint32_t kSlot = 2 * C::kThreads * 16;    // bytes per chunk slot
-  constexpr uint32_t kHalf = C::kThreads * 16;        // row g -> row g+8 within a slot
+  constexpr uint32_t kHalf = C::kThreads * 16;   // row g -> row g+8 within a slot
+  const uint32_t ring_lo = base + static_cast<uint32_t>(threadIdx.x * 16);
+  const uint32_t ring_hi = kDecHighBase - C::kSlotBytes + static_cast<uint32_t>(threadIdx.x * 16);
+  auto slot_addr = [&](int s) { return s == 0 ? ring_lo : ring_hi + static_cast<uint32_t>(s) * C::kSlotBytes; };
 
-  const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
+  const uint32_t lanesel = 0x00010000u | (static_cast<uint32_t>(lane) << 2);
   const int g = lane >> 2, tig = lane & 3;
   const int warps = gridDim.x * C::kWarps;
   const int tok_per_task = 8 * NG;
   const uint4 zero = make_uint4(0, 0, 0, 0);
 
-  // producer cursor: (task, chunk) running kDecDepth chunks ahead, across tasks
-  int p_task = blockIdx.x * C::kWarps + wid, p_ch = 0;
-  DecTask pd;
-  if (p_task < G.total_tasks) pd = dec_task(G, p_task, tok_per_task);
+  // producer cursor: (task, chunk) running kDecDepth - 1 chunks ahead, across tasks
+  int p_task = blockIdx.x * C::kWarps + wid;
+  const uint8_t* p_src = nullptr;   // this thread's 16 code bytes of row n0 + g, next chunk
+  int64_t p_kb = 0;                 // code bytes per row
+  int p_left = 0;                   // chunks left in the producer's task
+  bool p_tail_ok = true;            // this thread's part of a partial last chunk is in range
+  auto p_start = [&]() {
+    if (p_task < G.total_tasks) {
+      const DecTask d = dec_task(G, p_task, tok_per_task);
+      p_kb = d.P->k_in >> 2;
+      p_src = d.P->codes + static_cast<int64_t>(d.n0 + g) * p_kb + tig * 16;
+      p_left = d.nch;
+      const int rem = d.P->k_in & 255;
+      p_tail_ok = rem == 0 || 64 * tig < rem;
+    }
+  };
+  p_start();
   int issued = 0;
   auto produce_one = [&]() {   // always commits one group (empty past the end)
     if (p_task < G.total_tasks) {
-      const int kb = pd.P->k_in >> 2;
-      const bool valid = p_ch * 256 + 64 * tig < pd.P->k_in;
-      const uint8_t* src = pd.P->codes + static_cast<int64_t>(pd.n0 + g) * kb + p_ch * 64 + tig * 16;
-      const uint32_t dst = ring + static_cast<uint32_t>(issued % kDecDepth) * kSlot;
-      cp_async16(dst, valid ? src : pd.P->codes, valid);
-      cp_async16(dst + kHalf, valid ? src + 8 * static_cast<int64_t>(kb) : pd.P->codes, valid);
-      if (++p_ch == pd.nch) {
-        p_ch = 0;
+      const bool valid = p_left > 1 || p_tail_ok;
+      const uint32_t dst = slot_addr(issued % kDecDepth);
+      cp_async16(dst, valid ? p_src : G.p[0].codes, valid);
+      cp_async16(dst + kHalf, valid ? p_src + 8 * p_kb : G.p[0].codes, valid);
+      p_src += 64;
+      if (--p_left == 0) {
         p_task += warps;
-        if (p_task < G.total_tasks) pd = dec_task(G, p_task, tok_per_task);
+        p_start();
       }
     }
     cp_async_commit();
@@ -256,24 +284,40 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
     for (int k = 0; k < DecAcc<NG>::kSets; ++k)
 #pragma unroll
       for (int j = 0; j < NG; ++j) accs.v[k][j][0] = accs.v[k][j][1] = accs.v[k][j][2] = accs.v[k][j][3] = 0;
-    for (int ch = 0; ch < d.nch; ++ch) {
+    auto next_codes = [&](uint4& c0, uint4& c1) {
       produce_one();                      // chunk consumed + kDecDepth - 1
       cp_async_wait<kDecDepth - 1>();     // chunk `consumed` has landed (own copies only)
-      const uint32_t slot = ring + static_cast<uint32_t>(consumed % kDecDepth) * kSlot;
-      uint4 c0, c1;
+      const uint32_t slot = slot_addr(consumed % kDecDepth);
       asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(c0.x), "=r"(c0.y), "=r"(c0.z), "=r"(c0.w) : "r"(slot));
       asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w)
                    : "r"(slot + kHalf));
       ++consumed;
-      const bool mine = ch * 256 + 64 * tig < K;
+    };
+    const int nfull = K >> 8;
+    for (int ch = 0; ch < nfull; ++ch) {   // full chunks: every thread's 64 weights are in range
+      uint4 c0, c1;
+      next_codes(c0, c1);
       uint4 xv[NG][4];
 #pragma unroll
       for (int j = 0; j < NG; ++j) {
         const uint4* xp = reinterpret_cast<const uint4*>(xrow[j] + ch * 256);
 #pragma unroll
+        for (int q = 0; q < 4; ++q) xv[j][q] = __ldg(xp + q);
+      }
+      decode_chunk<NG>(accs, lanesel, c0, c1, xv);
+    }
+    if (K & 255) {   // partial last chunk: threads past the end use zero activations
+      uint4 c0, c1;
+      next_codes(c0, c1);
+      const bool mine = nfull * 256 + 64 * tig < K;
+      uint4 xv[NG][4];
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        const uint4* xp = reinterpret_cast<const uint4*>(xrow[j] + nfull * 256);
+#pragma unroll
         for (int q = 0; q < 4; ++q) xv[j][q] = mine ? __ldg(xp + q) : zero;
       }
-      decode_chunk<NG>(accs, lut, lane4, c0, c1, xv);
+      decode_chunk<NG>(accs, lanesel, c0, c1, xv);
     }
     int acc[NG][4];
 #pragma unroll

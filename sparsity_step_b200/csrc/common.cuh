@@ -24,6 +24,7 @@ enum : unsigned int {
   DEV_ST_TIMEOUT_MMA = 1u << 1,
   DEV_ST_TIMEOUT_EPILOGUE = 1u << 2,
   DEV_ST_TIMEOUT_DRAIN = 1u << 3,
+  DEV_ST_SMEM_LAYOUT = 1u << 4,   // a kernel found its shared memory at an unexpected address and did nothing
 };
 
 // A wait that has not completed after this long gives up (the longest legitimate
