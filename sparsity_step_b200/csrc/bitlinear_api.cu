@@ -9,6 +9,7 @@
 #include "../../include/bitlinear.h"
 #include "act_quant.cuh"
 #include "codes_kernels.cuh"
+#include "codes_tc.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
@@ -175,10 +176,56 @@ bl_status launch_fwd_codes_ng(const bl::FwdGroup& grp, cudaStream_t st) {
 }
 
 // Problems are already validated. Builds the task table in kernel parameters.
+// Tensor-core product from codes: up to 128 tokens per task, 128 weight rows.
+bl_status launch_fwd_codes_tc(const bl_fwd_problem* problems, int count, bool y_f32, cudaStream_t st) {
+  static thread_local bl::FwdGroup grp;
+  int64_t tasks = 0;
+  int n = 0;
+  for (int i = 0; i < count; ++i) {
+    const bl_fwd_problem& q = problems[i];
+    if (q.t == 0) continue;
+    bl::FwdProblem& d = grp.p[n++];
+    d.codes = q.codes;
+    d.xq = q.xq;
+    d.absmax = q.absmax;
+    d.w_scale = q.w_scale;
+    d.y = q.y_out;
+    d.acc = q.acc_out;
+    d.t = static_cast<int>(q.t);
+    d.k_in = static_cast<int>(q.k_in);
+    d.n_out = static_cast<int>(q.n_out);
+    d.task_begin = static_cast<int>(tasks);
+    const int64_t nt = q.t < bl::kTcMaxN ? (q.t + 15) / 16 * 16 : bl::kTcMaxN;
+    d.n_tile = static_cast<int>(nt);
+    tasks += ((q.n_out + bl::kTcRows - 1) / bl::kTcRows) * ((q.t + nt - 1) / nt);
+    if (tasks > INT32_MAX) return fail(BL_ERR_UNSUPPORTED_SHAPE, "too much work in one call");
+  }
+  grp.count = n;
+  grp.total_tasks = static_cast<int>(tasks);
+  grp.y_f32 = y_f32 ? 1 : 0;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(bl::fwd_codes_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         bl::kTcSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(codes tc)");
+    attr_set = true;
+  }
+  const int64_t blocks = tasks < device_sm_count() ? tasks : device_sm_count();
+  bl::fwd_codes_tc_kernel<<<static_cast<unsigned>(blocks), bl::kTcThreads, bl::kTcSmemBytes, st>>>(grp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "codes tc launch");
+  return BL_OK;
+}
+
+// Token batches of at least this many tokens (the largest in a call) take the
+// tensor-core product from codes; smaller ones the warp-MMA kernel.
+constexpr int64_t kCodesTcMinTokens = 16;
+
 bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32, cudaStream_t st) {
   int64_t tmax = 0;
   for (int i = 0; i < count; ++i) tmax = problems[i].t > tmax ? problems[i].t : tmax;
   if (tmax == 0) return BL_OK;
+  if (tmax >= kCodesTcMinTokens) return launch_fwd_codes_tc(problems, count, y_f32, st);
   const int ng = tmax <= 8 ? 1 : (tmax <= 16 ? 2 : 4);
   static thread_local bl::FwdGroup grp;   // ~16 KB: kept off the stack
   int64_t tasks = 0;

@@ -66,6 +66,7 @@ struct FwdProblem {
   int32_t* acc;            // [t, n_out] or null
   int t, k_in, n_out;
   int task_begin;          // first task index of this problem
+  int n_tile;              // tokens per task (tensor-core kernel only)
 };
 
 struct FwdGroup {
@@ -294,15 +295,30 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
       ++consumed;
     };
     const int nfull = K >> 8;
-    for (int ch = 0; ch < nfull; ++ch) {   // full chunks: every thread's 64 weights are in range
+    // full chunks: every thread's 64 weights are in range; the activations of the next
+    // chunk are loaded while this one is decoded
+    uint4 xn[NG][4];
+    if (nfull > 0) {
+#pragma unroll
+      for (int j = 0; j < NG; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xn[j][q] = __ldg(reinterpret_cast<const uint4*>(xrow[j]) + q);
+    }
+    for (int ch = 0; ch < nfull; ++ch) {
       uint4 c0, c1;
       next_codes(c0, c1);
       uint4 xv[NG][4];
 #pragma unroll
-      for (int j = 0; j < NG; ++j) {
-        const uint4* xp = reinterpret_cast<const uint4*>(xrow[j] + ch * 256);
+      for (int j = 0; j < NG; ++j)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) xv[j][q] = __ldg(xp + q);
+        for (int q = 0; q < 4; ++q) xv[j][q] = xn[j][q];
+      if (ch + 1 < nfull) {
+#pragma unroll
+        for (int j = 0; j < NG; ++j) {
+          const uint4* xp = reinterpret_cast<const uint4*>(xrow[j] + (ch + 1) * 256);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) xn[j][q] = __ldg(xp + q);
+        }
       }
       decode_chunk<NG>(accs, lanesel, c0, c1, xv);
     }

@@ -59,15 +59,6 @@ struct GemmArgs {
   const float* w_scale;      // gamma (EPI_FWD, EPI_GRADX)
 };
 
-__device__ __forceinline__ bool mbar_wait_plain(uint32_t bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
-  }
-  return true;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
