@@ -191,11 +191,11 @@ __device__ __forceinline__ DecTask dec_task(const FwdGroup& G, int task, int tok
   return d;
 }
 
-// 16-byte async copy global -> shared; `valid` false writes zeros (src not read).
+// 16-byte async copy global -> shared; `valid` false writes zeros (src not read). No
+// compiler memory barrier: ordering comes from the commit and wait that follow.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
-               "r"(valid ? 16 : 0)
-               : "memory");
+               "r"(valid ? 16 : 0));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>

@@ -8,12 +8,12 @@
 //
 // Per task (one problem, 128 weight rows, up to 128 tokens) the product is computed
 // with the weights on M, so Y^T[n, t] = sum_k W[n, k] * Xq[t, k] accumulates in TMEM:
-//   warp 0      cp.async producer: per stage the task's codes [128 rows x 64 B] (256
+//   warps 0-1   cp.async producers: per stage the task's codes [128 rows x 64 B] (256
 //               weights of K) and activations [tokens x 256 B] into a shared-memory
 //               ring of 4 stages; completion through cp.async.mbarrier.arrive.
-//   warp 1      TMEM allocator and MMA issuer: 8 x tcgen05.mma kind::i8 per stage with
+//   warp 2      TMEM allocator and MMA issuer: 8 x tcgen05.mma kind::i8 per stage with
 //               A (M = 128, K = 32) from TMEM and B from shared memory (128B swizzle).
-//   warps 2-9   decoders and epilogue: thread = one weight row; code bytes become
+//   warps 3-10  decoders and epilogue: thread = one weight row; code bytes become
 //               int8x4 words through a per-lane table and are stored into the stage's
 //               A columns with tcgen05.st; after a task's last stage they read the
 //               accumulator and write y[t, n] = acc * (a_t / 127) * gamma.
@@ -31,8 +31,10 @@ constexpr int kTcStages = 4;
 constexpr int kTcCodeBytes = kTcRows * 64;                // 8 KB: 256 weights of 128 rows
 constexpr int kTcBSub = kTcMaxN * 128;                    // one 128-byte-wide K slice of B
 constexpr int kTcStageBytes = kTcCodeBytes + 2 * kTcBSub;  // 40 KB
+constexpr int kTcProdWarps = 2;
+constexpr int kTcMmaWarp = kTcProdWarps;
 constexpr int kTcDecWarps = 8;
-constexpr int kTcThreads = 64 + 32 * kTcDecWarps;
+constexpr int kTcThreads = 32 * (kTcProdWarps + 1 + kTcDecWarps);
 constexpr uint32_t kTcLutBytes = 256 * 128;               // entry e of lane l at 128*e + 4*l
 constexpr uint32_t kTcDCols = 128;                        // accumulator columns
 constexpr uint32_t kTcACols = 64;                         // A columns per stage (256 int8)
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_codes_tc_kernel(const __gri
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(full0 + 8u * s, 32);           // every producer lane's cp.async arrive
+      mbar_init(full0 + 8u * s, 32 * kTcProdWarps);   // every producer lane's cp.async arrive
       mbar_init(afull0 + 8u * s, kTcDecWarps);
       mbar_init(empty0 + 8u * s, 1);           // MMA commit
     }
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_codes_tc_kernel(const __gri
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kTcMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -159,38 +161,54 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_codes_tc_kernel(const __gri
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------- cp.async producer
+  if (warp < kTcProdWarps) {
+    // ------------------------------------------------------------- cp.async producers
+    // Producer warp pw copies, per stage, code rows (lane >> 2) + 8i and token rows
+    // (lane >> 4) + 2i for i = pw, pw + kTcProdWarps, ...; a lane's 16-byte column
+    // within a row never changes, so only row offsets advance.
+    const int pw = warp;
+    const int cc = lane & 3, crow0 = (lane >> 2) + 8 * pw;                 // codes
+    const uint32_t cswz = static_cast<uint32_t>((cc ^ ((lane >> 3) & 3)) << 4);
+    const int bc16 = lane & 15, brow0 = (lane >> 4) + 2 * pw;              // activations
+    const uint32_t bsub = static_cast<uint32_t>((bc16 >> 3) * kTcBSub);
+    const int bc = bc16 & 7;
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
     for (int task = blockIdx.x; task < G.total_tasks && ok; task += gridDim.x) {
       const TcTask d = tc_task(G, task);
-      const FwdProblem& P = *d.P;
-      const int kb = P.k_in >> 2;
+      const uint8_t* const codes = d.P->codes;
+      const int8_t* const xq = d.P->xq;
+      const int K = d.P->k_in, kb = K >> 2;
+      const int rows_valid = min(kTcRows, d.P->n_out - d.n0);
+      const int toks_valid = min(d.P->n_tile, d.P->t - d.t0);
+      const int n_tile = d.P->n_tile;
+      const uint8_t* csrc = codes + static_cast<int64_t>(d.n0 + crow0) * kb + cc * 16;
+      const int8_t* bsrc = xq + static_cast<int64_t>(d.t0 + brow0) * K + bc16 * 16;
+      const int64_t cstep = static_cast<int64_t>(8 * kTcProdWarps) * kb;
+      const int64_t bstep = static_cast<int64_t>(2 * kTcProdWarps) * K;
       for (int ch = 0; ch < d.nch; ++ch) {
         const bool got = mbar_wait(empty0 + 8u * s, ph ^ 1u, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
-        const uint32_t cdst = st_codes(s), bdst = st_b(s);
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {   // codes: 128 rows x 4 pieces of 16 B
-          const int p = lane + 32 * i, row = p >> 2, c = p & 3;
-          const int byte = ch * 64 + c * 16;
-          const bool valid = d.n0 + row < P.n_out && byte < kb;
-          const uint8_t* src = P.codes + static_cast<int64_t>(d.n0 + row) * kb + byte;
-          cp_async16(cdst + static_cast<uint32_t>(row * 64 + ((c ^ ((row >> 1) & 3)) << 4)), valid ? src : P.codes, valid);
+        const uint32_t cdst = st_codes(s) + cswz;
+        const bool ck = ch * 64 + cc * 16 < kb;
+        const uint8_t* src = csrc + ch * 64;
+#pragma unroll
+        for (int row = crow0; row < kTcRows; row += 8 * kTcProdWarps) {
+          const bool valid = ck && row < rows_valid;
+          cp_async16(cdst + static_cast<uint32_t>(row * 64), valid ? src : codes, valid);
+          src += cstep;
         }
-        const int npieces = P.n_tile * 16;
-        for (int p = lane; p < npieces; p += 32) {   // activations: tokens x 16 pieces of 16 B
-          const int row = p >> 4, c16 = p & 15, sub = c16 >> 3, c = c16 & 7;
-          const int k = ch * 256 + c16 * 16;
-          const bool valid = d.t0 + row < P.t && k < P.k_in;
-          const int8_t* src = P.xq + static_cast<int64_t>(d.t0 + row) * P.k_in + k;
-          cp_async16(bdst + static_cast<uint32_t>(sub * kTcBSub + row * 128 + ((c ^ (row & 7)) << 4)),
-                     valid ? static_cast<const void*>(src) : static_cast<const void*>(P.xq), valid);
+        const uint32_t bdst = st_b(s) + bsub;
+        const bool bk = ch * 256 + bc16 * 16 < K;
+        const int8_t* bs = bsrc + ch * 256;
+        for (int row = brow0; row < n_tile; row += 2 * kTcProdWarps) {
+          const bool valid = bk && row < toks_valid;
+          cp_async16(bdst + static_cast<uint32_t>(row * 128 + ((bc ^ (row & 7)) << 4)), valid ? bs : xq, valid);
+          bs += bstep;
         }
         cp_async_arrive_noinc(full0 + 8u * s);
         if (++s == kTcStages) {
@@ -204,7 +222,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_codes_tc_kernel(const __gri
       atomicOr(&g_device_status, DEV_ST_TIMEOUT_PRODUCER);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");   // no copy in flight when the thread exits
-  } else if (warp == 1) {
+  } else if (warp == kTcMmaWarp) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int s = 0;
@@ -251,7 +269,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_codes_tc_kernel(const __gri
     }
   } else {
     // ------------------------------------------------------------- decoders + epilogue
-    const int e = warp - 2, q = warp & 3, h = e >> 2;
+    const int e = warp - (kTcMmaWarp + 1), q = warp & 3, h = e >> 2;
     const int r = 32 * q + lane;                         // weight row in the task = TMEM lane
     const uint32_t lanebase = lut | (static_cast<uint32_t>(lane) << 2);
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
@@ -306,23 +324,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_codes_tc_kernel(const __gri
       }
       tc_fence_after_sync();
       const float gamma = *P.w_scale;
+      const float* const absmax = P.absmax;
+      void* const yout = P.y;
+      int32_t* const accout = P.acc;
+      const int n_out = P.n_out, n_tile = P.n_tile;
+      const int toks_valid = min(n_tile, P.t - d.t0);
       const int n = d.n0 + r;
-      const int half = P.n_tile >> 1;
-      for (int c0 = h * half; c0 < (h + 1) * half; c0 += 8) {
-        uint32_t a8[8];
-        tmem_ld_32x32b_x8(tmem_base + lane_off + static_cast<uint32_t>(c0), a8);
-        tmem_ld_wait();
+      const bool row_ok = n < n_out;
+      const bool y_f32 = G.y_f32 != 0;
+      const int half = n_tile >> 1;
+      for (int cb = h * half; cb < (h + 1) * half; cb += 32) {
+        // row scales of up to 32 token columns: lane j holds column cb + j
+        float rs_l = 0.0f;
+        if (cb + lane < (h + 1) * half && cb + lane < toks_valid)
+          rs_l = __fmul_rn(__fdiv_rn(absmax[d.t0 + cb + lane], 127.0f), gamma);
+        const int cend = min(cb + 32, (h + 1) * half);
+        for (int c0 = cb; c0 < cend; c0 += 8) {
+          uint32_t a8[8];
+          tmem_ld_32x32b_x8(tmem_base + lane_off + static_cast<uint32_t>(c0), a8);
+          tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int tok = d.t0 + c0 + j;
-          if (tok < P.t && n < P.n_out) {
-            const int acc = static_cast<int>(a8[j]);
-            const float rs = __fmul_rn(__fdiv_rn(P.absmax[tok], 127.0f), gamma);
-            const float y = __fmul_rn(static_cast<float>(acc), rs);
-            const int64_t off = static_cast<int64_t>(tok) * P.n_out + n;
-            if (G.y_f32) static_cast<float*>(P.y)[off] = y;
-            else static_cast<__nv_bfloat16*>(P.y)[off] = __float2bfloat16_rn(y);
-            if (P.acc != nullptr) P.acc[off] = acc;
+          for (int j = 0; j < 8; ++j) {
+            const float rs = __shfl_sync(0xffffffffu, rs_l, c0 - cb + j);
+            const int col = c0 + j;
+            if (col < toks_valid && row_ok) {
+              const int acc = static_cast<int>(a8[j]);
+              const float y = __fmul_rn(static_cast<float>(acc), rs);
+              const int64_t off = static_cast<int64_t>(d.t0 + col) * n_out + n;
+              if (y_f32) static_cast<float*>(yout)[off] = y;
+              else static_cast<__nv_bfloat16*>(yout)[off] = __float2bfloat16_rn(y);
+              if (accout != nullptr) accout[off] = acc;
+            }
           }
         }
       }
@@ -337,7 +369,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_codes_tc_kernel(const __gri
   }
 
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kTcMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, 512);
   }
