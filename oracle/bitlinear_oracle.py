@@ -300,6 +300,68 @@ def dequant_x(q: np.ndarray, absmax: np.ndarray) -> np.ndarray:
     return q.astype(np.float64) * (absmax.astype(np.float64)[:, None] / 127.0)
 
 
+def grad_x_int8_dy(dy_bits: np.ndarray, mcode: np.ndarray, gamma: np.float32,
+                   rows: np.ndarray | None = None) -> tuple[np.ndarray, np.ndarray, np.ndarray, np.ndarray]:
+    """grad_X with dY quantised per token to int8, as an exact integer product.
+
+    An approximation this library offers for the input gradient (the pages keep dY in
+    higher precision): dY is quantised with the same per-token absmax rule as the
+    activations (BitNet b1.58 2B4T article section 一), then multiplied with the
+    masked ternary codes exactly in integers (Sparse-BitNet article section 六: the
+    input gradient goes through the effective weight), then rescaled:
+        acc[t,k] = sum_n q_dy[t,n] * mcode[n,k],  grad_x ~ acc * (a_t / 127) * gamma.
+    Returns (acc int32, grad_x fp64, q_dy, a_dy). ``rows`` selects tokens.
+    """
+    dyr = dy_bits if rows is None else dy_bits[rows]
+    q, a = act_quant(dyr)
+    acc, y = fwd(q, a, mcode.T, gamma)
+    return acc, y, q, a
+
+
+# --------------------------------------------------------------------------- diagnostics
+
+HIST_BINS = 17   # [k/8, (k+1)/8) of gamma for k = 0..15, then [2, inf)
+
+
+def threshold_hist(w: np.ndarray, keep: np.ndarray, gamma: np.float32, m_group: int) -> dict:
+    """Where the N:M threshold falls relative to the ternary levels.
+
+    Follows: Sparse-BitNet article section 五 (threshold decoupling: each group of 8
+    gets a threshold that splits kept from dropped weights; in the 1.58-bit model it
+    stays in the near-zero "noise" region instead of cutting into weights that
+    matter).
+    reading: a group's threshold is the largest magnitude among its dropped weights,
+    measured in units of gamma; ``hist[k]`` counts the groups whose threshold r has
+    k/8 <= r < (k+1)/8 (k = 0..15) and ``hist[16]`` those with r >= 2, the bin decided
+    exactly (8|w| against k * gamma in fp64, both products exact). Groups with no
+    dropped weight (N = M) are not counted. ``dropped`` counts dropped weights and
+    ``dropped_core`` those whose ternary code is nonzero (|w| > gamma / 2, the
+    rounding rule of the ternary quantiser), i.e. weights the mask cut from the
+    +-1 levels.
+    """
+    a = np.abs(np.asarray(w, dtype=np.float32)).astype(np.float64)
+    rows, k = a.shape
+    groups = a.reshape(rows, k // m_group, m_group)
+    kept = np.asarray(keep, dtype=bool).reshape(rows, k // m_group, m_group)
+    g64 = float(gamma)
+    hist = np.zeros(HIST_BINS, dtype=np.int64)
+    dropped = 0
+    core = 0
+    for r in range(rows):
+        for gi in range(k // m_group):
+            drop_vals = groups[r, gi][~kept[r, gi]]
+            if drop_vals.size == 0:
+                continue
+            dropped += drop_vals.size
+            core += int(np.sum(2.0 * drop_vals > g64))
+            t = drop_vals.max()
+            b = 0
+            while b < HIST_BINS - 1 and 8.0 * t >= (b + 1) * g64:
+                b += 1
+            hist[b] += 1
+    return {"hist": hist, "dropped": dropped, "dropped_core": core}
+
+
 # --------------------------------------------------------------------------- whole layer
 
 def layer_step(w: np.ndarray, x_bits: np.ndarray, dy_bits: np.ndarray,

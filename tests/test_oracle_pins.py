@@ -394,3 +394,103 @@ def test_grad_w_dequant_option_matches_forward_input():
     assert np.all(np.abs(xd - O.bf16_to_f32(x)) <= 0.5 * a[:, None] / 127.0 * (1 + 1e-6))
     gw = O.grad_w(dy, x, x_deq=xd)
     assert np.allclose(gw, _loops_grad_w(O.bf16_to_f32(dy).astype(np.float64), xd), rtol=1e-12, atol=1e-15)
+
+
+# ----------------------------------------------------------------------- threshold diagnostic
+
+
+@pytest.mark.parametrize("n,m,key", [(6, 8, "6_8"), (4, 8, "4_8"), (2, 8, "2_8"), (2, 4, "2_4")])
+def test_hand_threshold_hist(n, m, key):
+    w = _w_example()
+    qm = O.quant_mask(w, n, m)
+    h = O.threshold_hist(w, qm["keep"], qm["gamma"], m)
+    want = np.zeros(O.HIST_BINS, dtype=np.int64)
+    for b in _ints(f"thr_bins_{key}"):
+        want[b] += 1
+    assert np.array_equal(h["hist"], want)
+    assert h["dropped"] == _ints(f"thr_dropped_{key}")[0]
+    assert h["dropped_core"] == _ints(f"thr_core_{key}")[0]
+
+
+@pytest.mark.parametrize("n,m", [(6, 8), (4, 8), (3, 8), (2, 8), (2, 4), (1, 4)])
+def test_threshold_is_the_next_largest_magnitude(n, m):
+    # With ties, which tied weight is dropped changes nothing: the group threshold is
+    # the (n+1)-th largest magnitude, found here by sorting, without the mask.
+    w = _tied_weights(11, 6, 64)
+    qm = O.quant_mask(w, n, m)
+    h = O.threshold_hist(w, qm["keep"], qm["gamma"], m)
+    a = np.sort(np.abs(w).astype(np.float64).reshape(-1, m), axis=1)[:, ::-1]
+    thr = a[:, n]
+    g = float(qm["gamma"])
+    bins = np.array([min(16, sum(1 for k in range(1, 17) if 8.0 * t >= k * g)) for t in thr])
+    assert np.array_equal(h["hist"], np.bincount(bins, minlength=O.HIST_BINS))
+    groups = w.size // m
+    assert h["hist"].sum() == groups and h["dropped"] == groups * (m - n)
+    # dropped weights with a nonzero ternary code, counted from the codes themselves
+    assert h["dropped_core"] == int(np.sum((qm["code"] != 0) & ~qm["keep"].astype(bool)))
+
+
+def test_threshold_hist_8_8_is_empty():
+    w = synth.latent_weight(5, 8, 64)
+    qm = O.quant_mask(w, 8, 8)
+    h = O.threshold_hist(w, qm["keep"], qm["gamma"], 8)
+    assert h["hist"].sum() == 0 and h["dropped"] == 0 and h["dropped_core"] == 0
+
+
+def test_threshold_hist_bin_edges_inclusive():
+    # gamma = 1: a dropped magnitude of exactly k/8 opens bin k; one ulp below stays in k-1
+    for k in range(1, 17):
+        for val, want in ((np.float32(k / 8), k), (np.nextafter(np.float32(k / 8), np.float32(0)), k - 1)):
+            w = np.array([[4.0, 4.0, 4.0, 4.0, 4.0, 4.0, val, 0.0]], dtype=np.float32)
+            keep = np.array([[1, 1, 1, 1, 1, 1, 0, 0]], dtype=np.uint8)
+            h = O.threshold_hist(w, keep, np.float32(1.0), 8)
+            assert h["hist"][want] == 1, (k, float(val))
+
+
+# ----------------------------------------------------------------------- int8-dY input gradient
+
+
+def test_grad_x_int8_dy_brute_force():
+    rng = np.random.default_rng(21)
+    t, n, k = 3, 16, 8
+    dy = synth.f32_to_bf16_bits(rng.standard_normal((t, n)).astype(np.float32) * 0.01)
+    mcode = rng.integers(-1, 2, size=(n, k)).astype(np.int8)
+    gamma = np.float32(0.0375)
+    acc, y, q, a = O.grad_x_int8_dy(dy, mcode, gamma)
+    for ti in range(t):
+        for ki in range(k):
+            s = 0
+            for ni in range(n):
+                s += int(q[ti, ni]) * int(mcode[ni, ki])
+            assert acc[ti, ki] == s
+            assert y[ti, ki] == pytest.approx(s * float(a[ti]) / 127.0 * float(gamma), rel=1e-15, abs=0)
+
+
+def test_grad_x_int8_dy_exact_on_quantisation_grid():
+    # dY = q * 2^-e with |q| <= 127 and a 127 in each row: quantisation is lossless, so
+    # the integer path gives the exact input gradient
+    rng = np.random.default_rng(22)
+    t, n, k = 4, 64, 32
+    q = rng.integers(-127, 128, size=(t, n))
+    q[:, 0] = 127
+    dy = synth.f32_to_bf16_bits((q * 2.0 ** -9).astype(np.float32))
+    mcode = rng.integers(-1, 2, size=(n, k)).astype(np.int8)
+    gamma = np.float32(0.02)
+    _, y, qq, _ = O.grad_x_int8_dy(dy, mcode, gamma)
+    assert np.array_equal(qq, q)
+    assert np.allclose(y, O.grad_x(dy, mcode, gamma), rtol=1e-14, atol=0)
+
+
+def test_grad_x_int8_dy_error_within_quantisation_bound():
+    # each dY element moves by at most half a quantisation step a_t / 254 (plus the
+    # fp32 product's rounding), so |error| <= sum_n |c[n,k]| * gamma * a_t / 254 * (1 + 1e-6)
+    rng = np.random.default_rng(23)
+    t, n, k = 8, 256, 64
+    dy = synth.activation_bf16(31, t, n, std=1e-2, outliers=False)
+    mcode = rng.integers(-1, 2, size=(n, k)).astype(np.int8)
+    gamma = np.float32(0.03)
+    _, y, _, a = O.grad_x_int8_dy(dy, mcode, gamma)
+    exact = O.grad_x(dy, mcode, gamma)
+    bound = (np.abs(mcode).sum(axis=0)[None, :] * float(gamma) * a.astype(np.float64)[:, None] / 254.0) * (1 + 1e-6)
+    assert np.all(np.abs(y - exact) <= bound)
+    assert np.max(np.abs(y - exact)) > 0   # the approximation is not exact in general
