@@ -43,9 +43,9 @@ CFG_INDEX = 4   # the training-step workload's seed block
 # source has changed).
 TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum (1 pass) on the full-size
-    # grad_W launch (16384 x 2048 x 11008, CTA-pair kernel): 722,842,368 B read +
-    # 41,942,272 B written
-    "bwd_grad_w": {"sha": "e3829fad9d296712", "bytes": 764784640},
+    # grad_W launch (16384 x 2048 x 11008, CTA-pair kernel): 724,534,528 B read +
+    # 42,022,912 B written
+    "bwd_grad_w": {"sha": "e0f2f761070bdee5", "bytes": 766557440},
 }
 
 
@@ -662,6 +662,9 @@ def run_case(args) -> None:
     gx = torch.empty((t, k_in), dtype=torch.bfloat16, device=dev)
     gw = torch.empty((n_out, k_in), dtype=torch.bfloat16, device=dev)
     ws = torch.empty((B.bitlinear_bwd_workspace_size(t, k_in, n_out, True),), dtype=torch.uint8, device=dev)
+    ws_i8 = (torch.empty((B.bitlinear_grad_x_i8_workspace_size(t, k_in, n_out),), dtype=torch.uint8, device=dev)
+             if args.case == "grad_x_i8" else None)
+    hist = torch.empty((19,), dtype=torch.int64, device=dev)
     flops = 2.0 * t * k_in * n_out
     cases = {
         "quant_mask": (lambda: B.bitlinear_quant_mask(w, N_KEEP, M_GROUP, out=qm, workspace=qm["workspace"]),
@@ -673,6 +676,11 @@ def run_case(args) -> None:
         "grad_x": (lambda: B.bitlinear_bwd(dy, None, qm["codes"], qm["w_scale"], want_grad_w=False, grad_x=gx,
                                            workspace=ws, k_in=k_in), "TFLOP/s", flops),
         "grad_w": (lambda: B.bitlinear_bwd(dy, x, None, None, want_grad_x=False, grad_w=gw), "TFLOP/s", flops),
+        # int8-dY input gradient (an approximation; dY quantised per token): dense-equivalent ops
+        "grad_x_i8": (lambda: B.bitlinear_grad_x_i8(dy, qm["codes"], qm["w_scale"], k_in=k_in, grad_x=gx,
+                                                    workspace=ws_i8), "TOP/s", flops),
+        "mask_hist": (lambda: B.bitlinear_mask_threshold_hist(w, qm["mask"], qm["w_scale"], M_GROUP, out=hist),
+                      "GB/s", n_out * k_in * (4 + 1.0 / M_GROUP)),
     }
     fn, unit, work = cases[args.case]
     for _ in range(args.warmup):
@@ -808,7 +816,7 @@ SWEEP_SHAPES = {
                                    ("gate", 896, 4864), ("up", 896, 4864), ("down", 4864, 896)]),
     "qwen2.5-1.5b-mlp T=8192": (8192, [("gate", 1536, 8960), ("up", 1536, 8960), ("down", 8960, 1536)]),
 }
-SWEEP_NM = [(8, 8), (6, 8), (4, 8), (2, 4), (2, 8)]
+SWEEP_NM = [(8, 8), (6, 8), (4, 8), (3, 8), (2, 4), (2, 8)]
 
 
 def run_sweep(args) -> None:
@@ -865,7 +873,8 @@ def main(argv=None) -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=32, help="reference arm: tokens per sampled step")
     ap.add_argument("--ref-w-rows", type=int, default=64, help="reference arm: weight rows per sampled step")
-    ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_codes", "grad_x", "grad_w", "mma_peak_i8",
+    ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_codes", "grad_x", "grad_w", "grad_x_i8",
+                                       "mask_hist", "mma_peak_i8",
                              "mma_peak_bf16", "warp_mma_s8", "warp_mma_b1"],
                     help="time one kernel class alone on the --case-t/k/n shape")
     ap.add_argument("--case-t", type=int, default=TOKENS)

@@ -160,7 +160,8 @@ typedef struct {
  * Step a4 for up to 256 independent problems in one launch (e.g. every BitLinear of
  * a layer stack at one decode step, or the q/k/v or gate/up linears that share an
  * input). Same result as bitlinear_fwd with the codes operand for each problem; the
- * packed 2-bit codes are streamed once per 32 tokens. `problems` is a HOST array
+ * packed 2-bit codes are streamed once per 128 tokens (once per 8 or 16 tokens when
+ * the largest problem has fewer than 16). `problems` is a HOST array
  * (copied into the launch); y_dtype applies to all problems. Problems may have t = 0.
  * More than 256 problems: BL_ERR_UNSUPPORTED_SHAPE.
  */
@@ -184,6 +185,51 @@ size_t bitlinear_bwd_workspace_size(int64_t t, int64_t k_in, int64_t n_out, int 
 bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* codes, const float* w_scale, int64_t t,
                         int64_t k_in, int64_t n_out, uint16_t* grad_x, void* grad_w, int grad_w_dtype,
                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace bitlinear_grad_x_i8 needs (0 for an empty problem). */
+size_t bitlinear_grad_x_i8_workspace_size(int64_t t, int64_t k_in, int64_t n_out);
+
+/*
+ * Step a5 with dY quantised to int8: an approximation of the input gradient that runs
+ * on the int8 tensor cores. The pages keep the backward in higher precision; this
+ * entry point has no counterpart there (it is the library's faster variant, to be
+ * used only where its error is acceptable). dY is quantised per token exactly as
+ * bitlinear_act_quant quantises activations (BitNet b1.58 2B4T article, section 一),
+ * then multiplied with the masked ternary codes in integers (Sparse-BitNet article,
+ * section 六: the input gradient goes through the effective weight):
+ *   q, a   = act_quant(dy)                              ([t, n_out] int8, [t] fp32)
+ *   acc    = sum_n q[t, n] * masked_code[n, k]          (exact, int32)
+ *   grad_x = acc * (a_t / 127 * gamma)                  (fp32, then bf16)
+ * Each dY element moves by at most half a quantisation step, so
+ *   |grad_x - exact| <= sum_n |masked_code[n, k]| * gamma * a_t / 254  (+ rounding).
+ *
+ *   dy [t, n_out] bf16; codes [n_out, k_in / 4]; w_scale [1] gamma.
+ *   grad_x [t, k_in] bf16, out. acc_out [t, k_in] int32, out, nullable.
+ *   workspace bitlinear_grad_x_i8_workspace_size() bytes, 16-byte aligned (holds the
+ *   int8 dY, its absmax and the transposed int8 codes).
+ * Shapes as bitlinear_bwd, plus n_out % 64 == 0 (BL_ERR_UNSUPPORTED_SHAPE otherwise).
+ */
+bl_status bitlinear_grad_x_i8(const uint16_t* dy, const uint8_t* codes, const float* w_scale, int64_t t, int64_t k_in,
+                              int64_t n_out, uint16_t* grad_x, int32_t* acc_out, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
+ * Threshold-decoupling diagnostic (Sparse-BitNet article, section 五: the threshold
+ * that splits each group's kept from its dropped weights sits, for 1.58-bit weights,
+ * in the near-zero region rather than cutting weights that quantise to +-1).
+ *   For every group of m_group weights with at least one dropped weight (mask bit
+ *   clear), r = max |w| over its dropped weights / gamma:
+ *     hist_out[k]  (k = 0..15) counts groups with k/8 <= r < (k+1)/8,
+ *     hist_out[16] counts groups with r >= 2,
+ *     hist_out[17] = number of dropped weights,
+ *     hist_out[18] = dropped weights with a nonzero ternary code (|w| > gamma / 2).
+ *   Bin edges are decided exactly (8|w| against k * gamma in fp64).
+ *   w_latent [n_out, k_in] fp32, mask [n_out, k_in / m_group] (bit j = element j kept,
+ *   as written by bitlinear_quant_mask), w_scale [1] gamma, m_group 4 or 8.
+ *   hist_out: 19 uint64 on the device, 16-byte aligned, overwritten.
+ */
+bl_status bitlinear_mask_threshold_hist(const float* w_latent, const uint8_t* mask, const float* w_scale, int64_t n_out,
+                                        int64_t k_in, int m_group, unsigned long long* hist_out, void* stream);
 
 /* Synchronises the current device, then returns BL_OK; BL_ERR_TIMEOUT if a kernel
  * of this library gave up on a bounded wait since the last call (bits 0-3); or

@@ -13,6 +13,9 @@ from .bitlinear import (  # noqa: F401
     bitlinear_device_status,
     bitlinear_fwd,
     bitlinear_fwd_grouped,
+    bitlinear_grad_x_i8,
+    bitlinear_grad_x_i8_workspace_size,
+    bitlinear_mask_threshold_hist,
     bitlinear_quant_mask,
     bitlinear_quant_mask_noalloc,
     bitlinear_quant_mask_status,

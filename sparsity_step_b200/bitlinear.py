@@ -184,6 +184,46 @@ def bitlinear_bwd(dy: torch.Tensor, x: torch.Tensor | None, codes: torch.Tensor 
     return grad_x, grad_w
 
 
+def bitlinear_grad_x_i8_workspace_size(t: int, k_in: int, n_out: int) -> int:
+    return int(lib().bitlinear_grad_x_i8_workspace_size(t, k_in, n_out))
+
+
+def bitlinear_grad_x_i8(dy: torch.Tensor, codes: torch.Tensor, w_scale: torch.Tensor, *, k_in: int | None = None,
+                        grad_x: torch.Tensor | None = None, want_acc: bool = False,
+                        workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """Input gradient with dY quantised per token to int8 (an approximation); returns
+    {"grad_x", "acc" (or None)}."""
+    t, n_out = dy.shape
+    _need(dy, torch.bfloat16, None, "dy")
+    if k_in is None:
+        k_in = codes.shape[1] * 4
+    dev = dy.device
+    if grad_x is None:
+        grad_x = torch.empty((t, k_in), dtype=torch.bfloat16, device=dev)
+    acc = torch.empty((t, k_in), dtype=torch.int32, device=dev) if want_acc else None
+    need = bitlinear_grad_x_i8_workspace_size(t, k_in, n_out)
+    if workspace is None and need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    st = lib().bitlinear_grad_x_i8(_ptr(dy), _ptr(codes), _ptr(w_scale), t, k_in, n_out, _ptr(grad_x), _ptr(acc),
+                                   _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
+    check(st, "bitlinear_grad_x_i8")
+    return {"grad_x": grad_x, "acc": acc}
+
+
+def bitlinear_mask_threshold_hist(w: torch.Tensor, mask: torch.Tensor, w_scale: torch.Tensor, m_group: int, *,
+                                  out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Threshold-decoupling histogram: int64 [19] = 17 bins of max dropped |w| / gamma
+    (width 1/8, last bin >= 2), dropped weights, dropped weights with a nonzero code."""
+    n_out, k_in = w.shape
+    _need(w, torch.float32, None, "w")
+    if out is None:
+        out = torch.empty((19,), dtype=torch.int64, device=w.device)
+    st = lib().bitlinear_mask_threshold_hist(_ptr(w), _ptr(mask), _ptr(w_scale), n_out, k_in, m_group, _ptr(out),
+                                             _stream(stream))
+    check(st, "bitlinear_mask_threshold_hist")
+    return out
+
+
 def bitlinear_device_status() -> tuple[int, int]:
     """(status, bits): synchronise the device and read/clear the library's timeout bits."""
     bits = ctypes.c_uint(0)
@@ -199,5 +239,6 @@ __all__ = [
     "bitlinear_quant_mask_workspace_size", "bitlinear_quant_mask", "bitlinear_quant_mask_status",
     "bitlinear_quant_mask_noalloc",
     "bitlinear_act_quant", "bitlinear_fwd", "bitlinear_fwd_grouped", "bitlinear_bwd_workspace_size", "bitlinear_bwd",
+    "bitlinear_grad_x_i8_workspace_size", "bitlinear_grad_x_i8", "bitlinear_mask_threshold_hist",
     "bitlinear_device_status", "bitlinear_abi_version", "BL_OUT_BF16", "BL_OUT_F32", "_lib",
 ]

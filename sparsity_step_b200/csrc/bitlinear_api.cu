@@ -11,6 +11,7 @@
 #include "codes_kernels.cuh"
 #include "codes_tc.cuh"
 #include "common.cuh"
+#include "diag_kernels.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
 #include "quant_mask.cuh"
@@ -226,7 +227,7 @@ bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32
   for (int i = 0; i < count; ++i) tmax = problems[i].t > tmax ? problems[i].t : tmax;
   if (tmax == 0) return BL_OK;
   if (tmax >= kCodesTcMinTokens) return launch_fwd_codes_tc(problems, count, y_f32, st);
-  const int ng = tmax <= 8 ? 1 : (tmax <= 16 ? 2 : 4);
+  const int ng = tmax <= 8 ? 1 : 2;   // batches of 16+ tokens took the tensor-core path above
   static thread_local bl::FwdGroup grp;   // ~16 KB: kept off the stack
   int64_t tasks = 0;
   int n = 0;
@@ -251,8 +252,7 @@ bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32
   grp.total_tasks = static_cast<int>(tasks);
   grp.y_f32 = y_f32 ? 1 : 0;
   if (ng == 1) return launch_fwd_codes_ng<1>(grp, st);
-  if (ng == 2) return launch_fwd_codes_ng<2>(grp, st);
-  return launch_fwd_codes_ng<4>(grp, st);
+  return launch_fwd_codes_ng<2>(grp, st);
 }
 
 // ------------------------------------------------------------------ quant_mask launches
@@ -318,6 +318,72 @@ int qm_blocks(int64_t numel) {
   return static_cast<int>(b);
 }
 
+// Launch of the act_quant kernels (arguments already checked).
+bl_status enqueue_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t* xq_out, float* absmax_out,
+                            cudaStream_t st) {
+  const int k8 = static_cast<int>(k_in / 8);
+  const uint4* xv = reinterpret_cast<const uint4*>(x);
+  const unsigned g1 = static_cast<unsigned>(t);
+  if (k8 <= 512) {   // k_in <= 4096: one warp per row
+    const int per_sm = k8 <= 128 ? 8 : (k8 <= 256 ? 4 : 2);   // resident 256-thread blocks (registers)
+    int64_t blocks = (t + 7) / 8;
+    const int64_t cap = int64_t(device_sm_count()) * per_sm;
+    if (blocks > cap) blocks = cap;
+    const unsigned gb = static_cast<unsigned>(blocks);
+    if (k8 <= 128) bl::act_quant_warp_kernel<4><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (k8 <= 256) bl::act_quant_warp_kernel<8><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else bl::act_quant_warp_kernel<16><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+  } else {   // one CTA per row
+    const int vpt = (k8 + 255) / 256;
+    if (vpt <= 4) bl::act_quant_kernel<4, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (vpt <= 6) bl::act_quant_kernel<6, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (vpt <= 8) bl::act_quant_kernel<8, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (vpt <= 12) bl::act_quant_kernel<12, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else if (vpt <= 16) bl::act_quant_kernel<16, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    else bl::act_quant_long_kernel<<<g1, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  return BL_OK;
+}
+
+// The int8 tensor-core product y = (xq . w_i8^T) * (absmax / 127 * gamma) with w_i8
+// [n_out, k_in] K-major (arguments already checked).
+bl_status enqueue_fwd_i8(const int8_t* xq, const float* absmax, const int8_t* w_i8, const float* w_scale, int64_t t,
+                         int64_t k_in, int64_t n_out, int32_t* acc_out, void* y_out, bool y_f32, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (bl_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, k_in, t, 128, bl::kBM)) return s;
+  if (bl_status s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_i8, k_in, n_out, 128, bl::kBN)) return s;
+  bl::GemmArgs g{};
+  g.M = static_cast<int>(t);
+  g.N = static_cast<int>(n_out);
+  g.num_k_blocks = static_cast<int>((k_in + 127) / 128);
+  g.num_m_blocks = static_cast<int>((t + bl::kBM - 1) / bl::kBM);
+  g.num_n_blocks = static_cast<int>((n_out + bl::kBN - 1) / bl::kBN);
+  g.out = y_out;
+  g.out_f32 = y_f32 ? 1 : 0;
+  g.acc_out = acc_out;
+  g.row_absmax = absmax;
+  g.w_scale = w_scale;
+  if (acc_out) {   // int32 accumulators requested: per-row direct stores of y and acc
+    return launch_gemm<true, false, false, bl::EPI_FWD, false>(ta, tb, ta, g, st);
+  }
+  CUtensorMap to;
+  if (bl_status s = make_out_map(&to, y_out, t, n_out, g.out_f32)) return s;
+  if (use_cta_pair(t)) {   // each CTA of a pair loads 128 of the tile's 256 weight rows
+    CUtensorMap tb2;
+    if (bl_status s = make_map(&tb2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_i8, k_in, n_out, 128, 128)) return s;
+    bl::GemmArgs g2 = g;
+    g2.num_m_blocks = static_cast<int>((t + 255) / 256);
+    bool launched = false;
+    if (bl_status s = launch_gemm2<true, false, false, bl::EPI_FWD>(ta, tb2, to, g2, st, &launched)) return s;
+    if (launched) return BL_OK;
+  }
+  return launch_gemm<true, false, false, bl::EPI_FWD, true>(ta, tb, to, g, st);
+}
+
+inline size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+
 }  // namespace
 
 extern "C" {
@@ -370,31 +436,7 @@ bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t
   if (!x || !xq_out || !absmax_out) return fail(BL_ERR_INVALID_ARG, "x, xq_out, absmax_out are required");
   if (!aligned16(x) || !aligned16(xq_out) || !aligned16(absmax_out))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
-  cudaStream_t st = as_stream(stream);
-  const int k8 = static_cast<int>(k_in / 8);
-  const uint4* xv = reinterpret_cast<const uint4*>(x);
-  const unsigned g1 = static_cast<unsigned>(t);
-  if (k8 <= 512) {   // k_in <= 4096: one warp per row
-    const int per_sm = k8 <= 128 ? 8 : (k8 <= 256 ? 4 : 2);   // resident 256-thread blocks (registers)
-    int64_t blocks = (t + 7) / 8;
-    const int64_t cap = int64_t(device_sm_count()) * per_sm;
-    if (blocks > cap) blocks = cap;
-    const unsigned gb = static_cast<unsigned>(blocks);
-    if (k8 <= 128) bl::act_quant_warp_kernel<4><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-    else if (k8 <= 256) bl::act_quant_warp_kernel<8><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-    else bl::act_quant_warp_kernel<16><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-  } else {   // one CTA per row
-    const int vpt = (k8 + 255) / 256;
-    if (vpt <= 4) bl::act_quant_kernel<4, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-    else if (vpt <= 6) bl::act_quant_kernel<6, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-    else if (vpt <= 8) bl::act_quant_kernel<8, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-    else if (vpt <= 12) bl::act_quant_kernel<12, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-    else if (vpt <= 16) bl::act_quant_kernel<16, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-    else bl::act_quant_long_kernel<<<g1, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
-  }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
-  return BL_OK;
+  return enqueue_act_quant(x, t, k_in, xq_out, absmax_out, as_stream(stream));
 }
 
 bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* codes, const int8_t* w_i8,
@@ -412,37 +454,7 @@ bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* co
   if (!aligned16(xq) || !aligned16(absmax) || !aligned16(y_out) || (acc_out && !aligned16(acc_out)))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
   cudaStream_t st = as_stream(stream);
-  if (w_i8) {
-    CUtensorMap ta, tb;
-    if (bl_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, k_in, t, 128, bl::kBM)) return s;
-    if (bl_status s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_i8, k_in, n_out, 128, bl::kBN)) return s;
-    bl::GemmArgs g{};
-    g.M = static_cast<int>(t);
-    g.N = static_cast<int>(n_out);
-    g.num_k_blocks = static_cast<int>((k_in + 127) / 128);
-    g.num_m_blocks = static_cast<int>((t + bl::kBM - 1) / bl::kBM);
-    g.num_n_blocks = static_cast<int>((n_out + bl::kBN - 1) / bl::kBN);
-    g.out = y_out;
-    g.out_f32 = y_dtype == BL_OUT_F32;
-    g.acc_out = acc_out;
-    g.row_absmax = absmax;
-    g.w_scale = w_scale;
-    if (acc_out) {   // int32 accumulators requested: per-row direct stores of y and acc
-      return launch_gemm<true, false, false, bl::EPI_FWD, false>(ta, tb, ta, g, st);
-    }
-    CUtensorMap to;
-    if (bl_status s = make_out_map(&to, y_out, t, n_out, g.out_f32)) return s;
-    if (use_cta_pair(t)) {   // each CTA of a pair loads 128 of the tile's 256 weight rows
-      CUtensorMap tb2;
-      if (bl_status s = make_map(&tb2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_i8, k_in, n_out, 128, 128)) return s;
-      bl::GemmArgs g2 = g;
-      g2.num_m_blocks = static_cast<int>((t + 255) / 256);
-      bool launched = false;
-      if (bl_status s = launch_gemm2<true, false, false, bl::EPI_FWD>(ta, tb2, to, g2, st, &launched)) return s;
-      if (launched) return BL_OK;
-    }
-    return launch_gemm<true, false, false, bl::EPI_FWD, true>(ta, tb, to, g, st);
-  }
+  if (w_i8) return enqueue_fwd_i8(xq, absmax, w_i8, w_scale, t, k_in, n_out, acc_out, y_out, y_dtype == BL_OUT_F32, st);
   bl_fwd_problem prob{xq, absmax, codes, w_scale, t, k_in, n_out, acc_out, y_out};
   return launch_fwd_codes(&prob, 1, y_dtype == BL_OUT_F32, st);
 }
@@ -554,6 +566,63 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* co
     if (!launched)
       if (bl_status s = launch_gemm<false, true, true, bl::EPI_GRADW, true>(ta, tb, to, g, st)) return s;
   }
+  return BL_OK;
+}
+
+size_t bitlinear_grad_x_i8_workspace_size(int64_t t, int64_t k_in, int64_t n_out) {
+  if (t <= 0 || k_in <= 0 || n_out <= 0) return 0;
+  return round256(static_cast<size_t>(t) * n_out) + round256(static_cast<size_t>(t) * 4) +
+         static_cast<size_t>(k_in) * static_cast<size_t>(n_out);
+}
+
+bl_status bitlinear_grad_x_i8(const uint16_t* dy, const uint8_t* codes, const float* w_scale, int64_t t, int64_t k_in,
+                              int64_t n_out, uint16_t* grad_x, int32_t* acc_out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  if (!codes || !w_scale) return fail(BL_ERR_INVALID_ARG, "codes and w_scale are required");
+  if (bl_status s = check_shape(t, k_in, n_out)) return s;
+  if (n_out % 64) return fail(BL_ERR_UNSUPPORTED_SHAPE, "n_out=%lld: the int8-dY gradient needs n_out %% 64 == 0", (long long)n_out);
+  if (!aligned16(codes) || !aligned16(w_scale)) return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  if (t == 0) return BL_OK;
+  if (!dy || !grad_x) return fail(BL_ERR_INVALID_ARG, "dy and grad_x are required");
+  if (!aligned16(dy) || !aligned16(grad_x) || (acc_out && !aligned16(acc_out)) || (workspace && !aligned16(workspace)))
+    return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  const size_t need = bitlinear_grad_x_i8_workspace_size(t, k_in, n_out);
+  if (!workspace || workspace_bytes < need) return fail(BL_ERR_WORKSPACE, "workspace too small: %zu < %zu", workspace_bytes, need);
+  cudaStream_t st = as_stream(stream);
+  int8_t* dyq = static_cast<int8_t*>(workspace);
+  float* a = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256(static_cast<size_t>(t) * n_out));
+  int8_t* ct = static_cast<int8_t*>(workspace) + round256(static_cast<size_t>(t) * n_out) + round256(static_cast<size_t>(t) * 4);
+  if (bl_status s = enqueue_act_quant(dy, t, n_out, dyq, a, st)) return s;
+  const dim3 grid(static_cast<unsigned>((n_out + 63) / 64), static_cast<unsigned>(k_in / 64));
+  bl::expand_codes_t_i8_kernel<<<grid, 256, 0, st>>>(codes, static_cast<int>(n_out), static_cast<int>(k_in), ct);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "transpose-expand launch");
+  // grad_x[t, k] = sum_n dyq[t, n] * C^T[k, n], rescaled by a_t / 127 * gamma
+  return enqueue_fwd_i8(dyq, a, ct, w_scale, t, n_out, k_in, acc_out, grad_x, false, st);
+}
+
+bl_status bitlinear_mask_threshold_hist(const float* w_latent, const uint8_t* mask, const float* w_scale, int64_t n_out,
+                                        int64_t k_in, int m_group, unsigned long long* hist_out, void* stream) {
+  g_err[0] = 0;
+  if (!w_latent || !mask || !w_scale || !hist_out) return fail(BL_ERR_INVALID_ARG, "w_latent, mask, w_scale, hist_out are required");
+  if (m_group != 4 && m_group != 8) return fail(BL_ERR_INVALID_ARG, "m_group must be 4 or 8");
+  if (bl_status s = check_shape(0, k_in, n_out)) return s;
+  if (!aligned16(w_latent) || !aligned16(w_scale) || !aligned16(hist_out))
+    return fail(BL_ERR_ALIGNMENT, "w_latent, w_scale and hist_out must be 16-byte aligned");
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e = cudaMemsetAsync(hist_out, 0, bl::kHistWords * sizeof(unsigned long long), st);
+  if (e != cudaSuccess) return cuda_fail(e, "histogram clear");
+  const int64_t ngroups = n_out * k_in / m_group;
+  int64_t blocks = (ngroups + 255) / 256;
+  const int64_t cap = int64_t(device_sm_count()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (m_group == 8)
+    bl::threshold_hist_kernel<8><<<static_cast<unsigned>(blocks), 256, 0, st>>>(w_latent, mask, w_scale, ngroups, hist_out);
+  else
+    bl::threshold_hist_kernel<4><<<static_cast<unsigned>(blocks), 256, 0, st>>>(w_latent, mask, w_scale, ngroups, hist_out);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "histogram launch");
   return BL_OK;
 }
 

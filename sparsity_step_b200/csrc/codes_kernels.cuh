@@ -201,7 +201,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int NG>   // token groups of 8 per task (1, 2 or 4)
+template <int NG>   // token groups of 8 per task (1 or 2)
 __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(const __grid_constant__ FwdGroup G) {
   using C = DecCfg<NG>;
   extern __shared__ __align__(1024) uint8_t dsmem[];

@@ -119,6 +119,27 @@ def test_bwd_validation(L):
     assert L.bitlinear_bwd(GOOD, BAD, None, None, 16, 896, 896, None, GOOD, 0, None, 0, None) == -3
 
 
+def test_grad_x_i8_validation(L):
+    need = L.bitlinear_grad_x_i8_workspace_size(16, 896, 2048)
+    assert need == 16 * 2048 + 256 + 896 * 2048
+    assert L.bitlinear_grad_x_i8_workspace_size(0, 896, 2048) == 0
+    # n_out must be a multiple of 64 on this path
+    assert L.bitlinear_grad_x_i8(GOOD, GOOD, GOOD, 16, 896, 144, GOOD, None, GOOD, 1 << 30, None) == -2
+    # codes / w_scale required; workspace checked
+    assert L.bitlinear_grad_x_i8(GOOD, None, GOOD, 16, 896, 2048, GOOD, None, GOOD, need, None) == -1
+    assert L.bitlinear_grad_x_i8(GOOD, GOOD, GOOD, 16, 896, 2048, GOOD, None, GOOD, need - 16, None) == -7
+    assert L.bitlinear_grad_x_i8(GOOD, GOOD, GOOD, 16, 896, 2048, BAD, None, GOOD, need, None) == -3
+    # empty batch: nothing to do, the t-sized arrays may be NULL
+    assert L.bitlinear_grad_x_i8(None, GOOD, GOOD, 0, 896, 2048, None, None, None, 0, None) == 0
+
+
+def test_mask_threshold_hist_validation(L):
+    assert L.bitlinear_mask_threshold_hist(GOOD, GOOD, GOOD, 896, 896, 6, GOOD, None) == -1
+    assert L.bitlinear_mask_threshold_hist(None, GOOD, GOOD, 896, 896, 8, GOOD, None) == -1
+    assert L.bitlinear_mask_threshold_hist(GOOD, GOOD, GOOD, 896, 100, 8, GOOD, None) == -2
+    assert L.bitlinear_mask_threshold_hist(GOOD, GOOD, GOOD, 896, 896, 8, BAD, None) == -3
+
+
 def test_last_error_is_thread_local_message(L):
     assert L.bitlinear_act_quant(None, 4, 896, GOOD, GOOD, None) == -1
     assert "required" in _err(L)

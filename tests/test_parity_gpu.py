@@ -123,7 +123,7 @@ def test_config2_qwen05_linears(idx):
 QWEN15_MLP = [("gate", 1536, 8960), ("up", 1536, 8960), ("down", 8960, 1536)]
 
 
-@pytest.mark.parametrize("nm", [(8, 8), (6, 8), (4, 8), (2, 4), (2, 8)], ids=lambda v: f"{v[0]}of{v[1]}")
+@pytest.mark.parametrize("nm", [(8, 8), (6, 8), (4, 8), (3, 8), (2, 4), (2, 8)], ids=lambda v: f"{v[0]}of{v[1]}")
 @pytest.mark.parametrize("idx", range(3), ids=[s[0] for s in QWEN15_MLP])
 def test_config3_nm_sweep(idx, nm):
     _, k_in, n_out = QWEN15_MLP[idx]
@@ -292,3 +292,79 @@ def test_range_error_reported():
 def test_no_device_timeouts():
     st, bits = B.bitlinear_device_status()
     assert st == 0 and bits == 0
+
+
+# ------------------------------------------------------------------ diagnostics and the int8-dY gradient
+
+
+def _hist_by_sorting(w, gamma, n, m):
+    """Threshold histogram from sorted magnitudes (the (n+1)-th largest |w| of each
+    group), vectorised; equal to the oracle's threshold_hist by the CPU pins."""
+    a = np.sort(np.abs(w).astype(np.float64).reshape(-1, m), axis=1)[:, ::-1]
+    g = float(gamma)
+    if n == m:
+        return np.zeros(O.HIST_BINS, np.int64), 0, 0
+    thr = a[:, n]
+    b = np.zeros(thr.shape, np.int64)
+    for k in range(1, O.HIST_BINS):
+        b += (8.0 * thr >= k * g)
+    core = int(np.sum(2.0 * a[:, n:] > g))
+    return np.bincount(b, minlength=O.HIST_BINS), a.shape[0] * (m - n), core
+
+
+@pytest.mark.parametrize("nm", [(6, 8), (4, 8), (3, 8), (2, 8), (2, 4), (8, 8)])
+def test_threshold_hist_oracle(nm):
+    n, m = nm
+    w = synth.latent_weight(synth.config_seed(3, 60 + 10 * n + m), 192, 1536)
+    ref_qm = O.quant_mask(w, n, m)
+    ref = O.threshold_hist(w, ref_qm["keep"], ref_qm["gamma"], m)
+    qm = gpu_quant_mask(w, n, m)
+    h = B.bitlinear_mask_threshold_hist(f32_to_dev(w), qm["mask"], qm["w_scale"], m).cpu().numpy()
+    assert_exact(h[:O.HIST_BINS], ref["hist"], f"hist {n}:{m}")
+    assert h[O.HIST_BINS] == ref["dropped"] and h[O.HIST_BINS + 1] == ref["dropped_core"]
+
+
+@pytest.mark.parametrize("nm", [(6, 8), (2, 4)])
+def test_threshold_hist_full_size(nm):
+    # the training workload's gate weights, 11008 x 2048
+    n, m = nm
+    w = synth.latent_weight(synth.config_seed(4, 0), 11008, 2048)
+    qm = gpu_quant_mask(w, n, m)
+    gamma = qm["w_scale"].cpu().numpy()[0]
+    h = B.bitlinear_mask_threshold_hist(f32_to_dev(w), qm["mask"], qm["w_scale"], m).cpu().numpy()
+    hist, dropped, core = _hist_by_sorting(w, gamma, n, m)
+    assert_exact(h[:O.HIST_BINS], hist, f"full-size hist {n}:{m}")
+    assert h[O.HIST_BINS] == dropped and h[O.HIST_BINS + 1] == core
+
+
+@pytest.mark.parametrize("t,k_in,n_out", [(64, 896, 896), (300, 576, 1536), (1, 2048, 256)])
+def test_grad_x_int8_dy(t, k_in, n_out):
+    w, _, dy = layer_inputs(1, 70 + t, t, k_in, n_out)
+    ref_qm = O.quant_mask(w, 6, 8)
+    qm = gpu_quant_mask(w, 6, 8)
+    acc_ref, y_ref, _, _ = O.grad_x_int8_dy(dy, ref_qm["mcode"], ref_qm["gamma"])
+    dyd = bits_to_dev_bf16(dy)
+    out = B.bitlinear_grad_x_i8(dyd, qm["codes"], qm["w_scale"], k_in=k_in, want_acc=True)
+    torch.cuda.synchronize()
+    assert_exact(out["acc"].cpu().numpy(), acc_ref, f"grad_x_i8 acc {t}x{k_in}<-{n_out}")
+    assert_bf16_within_ulp(bf16_dev_to_bits(out["grad_x"]), y_ref, f"grad_x_i8 y (acc path)")
+    out2 = B.bitlinear_grad_x_i8(dyd, qm["codes"], qm["w_scale"], k_in=k_in)
+    torch.cuda.synchronize()
+    assert_bf16_within_ulp(bf16_dev_to_bits(out2["grad_x"]), y_ref, f"grad_x_i8 y")
+    # the approximation against the exact input gradient
+    exact = O.grad_x(dy, ref_qm["mcode"], ref_qm["gamma"])
+    assert np.max(np.abs(y_ref - exact)) <= 2e-2 * np.max(np.abs(exact))
+
+
+def test_grad_x_int8_dy_training_shape():
+    # down projection of the training workload (dY [16384, 2048] -> grad_x [16384, 11008]),
+    # sampled token rows against the oracle
+    t, k_in, n_out = 16384, 11008, 2048
+    w, _, dy = layer_inputs(4, 2, t, k_in, n_out)
+    ref_qm = O.quant_mask(w, 6, 8)
+    qm = gpu_quant_mask(w, 6, 8)
+    rows = sample_rows(t, 5)
+    acc_ref, y_ref, _, _ = O.grad_x_int8_dy(dy, ref_qm["mcode"], ref_qm["gamma"], rows=rows)
+    out = B.bitlinear_grad_x_i8(bits_to_dev_bf16(dy), qm["codes"], qm["w_scale"], k_in=k_in)
+    torch.cuda.synchronize()
+    assert_bf16_within_ulp(bf16_dev_to_bits(out["grad_x"])[rows], y_ref, "grad_x_i8 training shape")
