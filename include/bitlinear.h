@@ -160,8 +160,8 @@ typedef struct {
  * Step a4 for up to 256 independent problems in one launch (e.g. every BitLinear of
  * a layer stack at one decode step, or the q/k/v or gate/up linears that share an
  * input). Same result as bitlinear_fwd with the codes operand for each problem; the
- * packed 2-bit codes are streamed once per 128 tokens (once per 8 or 16 tokens when
- * the largest problem has fewer than 16). `problems` is a HOST array
+ * packed 2-bit codes are streamed once per 128 tokens (once per 8 tokens when the
+ * largest problem has at most 8). `problems` is a HOST array
  * (copied into the launch); y_dtype applies to all problems. Problems may have t = 0.
  * More than 256 problems: BL_ERR_UNSUPPORTED_SHAPE.
  */

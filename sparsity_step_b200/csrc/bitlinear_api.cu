@@ -218,16 +218,18 @@ bl_status launch_fwd_codes_tc(const bl_fwd_problem* problems, int count, bool y_
   return BL_OK;
 }
 
-// Token batches of at least this many tokens (the largest in a call) take the
-// tensor-core product from codes; smaller ones the warp-MMA kernel.
-constexpr int64_t kCodesTcMinTokens = 16;
+// Token batches of more than 8 tokens (the largest in a call) take the tensor-core
+// product from codes; up to 8 the warp-MMA kernel (one 8-token MMA column group).
+// Measured on the 36-layer decode stack: 12 tokens 0.526 ms on two warp-MMA column
+// groups against 0.38 ms for 16 tokens on the tensor cores.
+constexpr int64_t kCodesTcMinTokens = 9;
 
 bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32, cudaStream_t st) {
   int64_t tmax = 0;
   for (int i = 0; i < count; ++i) tmax = problems[i].t > tmax ? problems[i].t : tmax;
   if (tmax == 0) return BL_OK;
   if (tmax >= kCodesTcMinTokens) return launch_fwd_codes_tc(problems, count, y_f32, st);
-  const int ng = tmax <= 8 ? 1 : 2;   // batches of 16+ tokens took the tensor-core path above
+  constexpr int ng = 1;   // batches of 9+ tokens took the tensor-core path above
   static thread_local bl::FwdGroup grp;   // ~16 KB: kept off the stack
   int64_t tasks = 0;
   int n = 0;
@@ -251,8 +253,7 @@ bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32
   grp.count = n;
   grp.total_tasks = static_cast<int>(tasks);
   grp.y_f32 = y_f32 ? 1 : 0;
-  if (ng == 1) return launch_fwd_codes_ng<1>(grp, st);
-  return launch_fwd_codes_ng<2>(grp, st);
+  return launch_fwd_codes_ng<ng>(grp, st);
 }
 
 // ------------------------------------------------------------------ quant_mask launches

@@ -111,6 +111,42 @@ __device__ __forceinline__ uint32_t lut_lookup(uint32_t w, uint32_t lanesel) {
   return v;
 }
 
+// Sixteen codes (code j at bits 2j of w) -> four int8x4 words in natural order with byte
+// permutes only (no table): nibble m of (w & 0x33333333) holds code 2m and nibble m of
+// ((w >> 2) & 0x33333333) code 2m+1; as permute selectors into the bytes {0x00, 0x01,
+// 0x00, 0xFF} they decode the even and the odd codes, and two more permutes interleave
+// them. Same result as four table lookups (byte j of w -> o_j), on the ALU pipe instead of
+// the shared-memory pipe; the decode kernel uses it for some words to balance the two.
+__device__ __forceinline__ void decode16(uint32_t w, uint32_t& o0, uint32_t& o1, uint32_t& o2, uint32_t& o3) {
+  constexpr uint32_t kTable = 0xFF000100u;
+  const uint32_t ev = w & 0x33333333u, od = (w >> 2) & 0x33333333u;
+  const uint32_t e_lo = __byte_perm(kTable, 0u, ev), e_hi = __byte_perm(kTable, 0u, ev >> 16);
+  const uint32_t o_lo = __byte_perm(kTable, 0u, od), o_hi = __byte_perm(kTable, 0u, od >> 16);
+  o0 = __byte_perm(e_lo, o_lo, 0x5140u);   // codes 0..3
+  o1 = __byte_perm(e_lo, o_lo, 0x7362u);   // codes 4..7
+  o2 = __byte_perm(e_hi, o_hi, 0x5140u);   // codes 8..11
+  o3 = __byte_perm(e_hi, o_hi, 0x7362u);   // codes 12..15
+}
+
+// Which of a chunk's eight code words (bit 2h + r: word h of row half r) are decoded by
+// byte permutes rather than table lookups: two of eight (measured on B200: batch 1
+// 0.234 -> 0.224 ms per 36-layer step; all-table decoding is limited by the shared-memory
+// instruction queue, half-and-half by the ALU at batch 1).
+constexpr unsigned kDecPrmtWords = 0x22;
+
+template <bool kPrmt>
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t lanesel, uint32_t& o0, uint32_t& o1, uint32_t& o2,
+                                            uint32_t& o3) {
+  if (kPrmt) {
+    decode16(w, o0, o1, o2, o3);
+  } else {
+    o0 = lut_lookup<0>(w, lanesel);
+    o1 = lut_lookup<1>(w, lanesel);
+    o2 = lut_lookup<2>(w, lanesel);
+    o3 = lut_lookup<3>(w, lanesel);
+  }
+}
+
 // Accumulators per token group, optionally split into independent sets (summed at
 // the end) to shorten the MMA dependency chain; one set measured fastest because
 // the registers a split costs lower the number of resident warps.
@@ -121,31 +157,30 @@ struct DecAcc {
 };
 
 // Two MMA steps from one 32-bit word of each row's codes (bytes 0..3 = steps 2h, 2h+1).
-template <int NG>
+template <int NG, int H>
 __device__ __forceinline__ void decode_mma_word(DecAcc<NG>& acc, uint32_t lanesel, uint32_t w0, uint32_t w1,
-                                                const uint4 (&xv)[NG][4], int h) {
+                                                const uint4 (&xv)[NG][4]) {
   constexpr int S = DecAcc<NG>::kSets;
-  {   // step 2h: bytes 0 (a0) and 1 (a2) of row g's word, of row g+8's word (a1, a3)
-    const uint32_t a0 = lut_lookup<0>(w0, lanesel), a2 = lut_lookup<1>(w0, lanesel);
-    const uint32_t a1 = lut_lookup<0>(w1, lanesel), a3 = lut_lookup<1>(w1, lanesel);
+  uint32_t r0[4], r1[4];   // decoded words of row g (w0) and row g+8 (w1)
+  decode_word<((kDecPrmtWords >> (2 * H)) & 1u) != 0>(w0, lanesel, r0[0], r0[1], r0[2], r0[3]);
+  decode_word<((kDecPrmtWords >> (2 * H + 1)) & 1u) != 0>(w1, lanesel, r1[0], r1[1], r1[2], r1[3]);
+  // step 2h: bytes 0 (a0) and 1 (a2) of row g's word, of row g+8's word (a1, a3)
 #pragma unroll
-    for (int j = 0; j < NG; ++j) mma_m16n8k32_s8(acc.v[(2 * h) % S][j], a0, a1, a2, a3, xv[j][h].x, xv[j][h].y);
-  }
-  {   // step 2h+1: bytes 2, 3
-    const uint32_t a0 = lut_lookup<2>(w0, lanesel), a2 = lut_lookup<3>(w0, lanesel);
-    const uint32_t a1 = lut_lookup<2>(w1, lanesel), a3 = lut_lookup<3>(w1, lanesel);
+  for (int j = 0; j < NG; ++j)
+    mma_m16n8k32_s8(acc.v[(2 * H) % S][j], r0[0], r1[0], r0[1], r1[1], xv[j][H].x, xv[j][H].y);
+  // step 2h+1: bytes 2, 3
 #pragma unroll
-    for (int j = 0; j < NG; ++j) mma_m16n8k32_s8(acc.v[(2 * h + 1) % S][j], a0, a1, a2, a3, xv[j][h].z, xv[j][h].w);
-  }
+  for (int j = 0; j < NG; ++j)
+    mma_m16n8k32_s8(acc.v[(2 * H + 1) % S][j], r0[2], r1[2], r0[3], r1[3], xv[j][H].z, xv[j][H].w);
 }
 
 template <int NG>
 __device__ __forceinline__ void decode_chunk(DecAcc<NG>& acc, uint32_t lanesel, const uint4& c0, const uint4& c1,
                                              const uint4 (&xv)[NG][4]) {
-  decode_mma_word<NG>(acc, lanesel, c0.x, c1.x, xv, 0);
-  decode_mma_word<NG>(acc, lanesel, c0.y, c1.y, xv, 1);
-  decode_mma_word<NG>(acc, lanesel, c0.z, c1.z, xv, 2);
-  decode_mma_word<NG>(acc, lanesel, c0.w, c1.w, xv, 3);
+  decode_mma_word<NG, 0>(acc, lanesel, c0.x, c1.x, xv);
+  decode_mma_word<NG, 1>(acc, lanesel, c0.y, c1.y, xv);
+  decode_mma_word<NG, 2>(acc, lanesel, c0.z, c1.z, xv);
+  decode_mma_word<NG, 3>(acc, lanesel, c0.w, c1.w, xv);
 }
 
 // Per-thread streaming: each thread copies the 32 code bytes it will itself decode
@@ -201,7 +236,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int NG>   // token groups of 8 per task (1 or 2)
+template <int NG>   // token groups of 8 per task
 __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(const __grid_constant__ FwdGroup G) {
   using C = DecCfg<NG>;
   extern __shared__ __align__(1024) uint8_t dsmem[];

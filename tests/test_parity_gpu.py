@@ -160,7 +160,7 @@ def test_config5_decode_batches(idx, layer):
                   f32=(b == 8))
 
 
-@pytest.mark.parametrize("b", [1, 3, 8, 16, 32, 128])
+@pytest.mark.parametrize("b", [1, 3, 8, 12, 16, 32, 128])
 def test_config5_grouped_layer(b):
     """All seven linears of one layer in one grouped launch, mixed shapes."""
     probs, refs = [], []
@@ -196,7 +196,7 @@ def test_config5_prefill_8192(idx):
 # ------------------------------------------------------------------ edge cases
 
 
-@pytest.mark.parametrize("t", [1, 5, 127, 129, 300])
+@pytest.mark.parametrize("t", [1, 5, 12, 127, 129, 300])
 def test_ragged_token_counts(t):
     # k_in = 576 ends the int8 K loop on a half-filled 128-byte stage; n_out = 144
     # ends the bf16 reduction of grad_x on a partial 64-row stage and leaves a
