@@ -1,4 +1,6 @@
-// Tensor-pipe throughput probe (measurement only, not part of the BitLinear ABI):
+// Probes (measurement and self-tests only, not part of the BitLinear ABI).
+//
+// Tensor-pipe throughput probe:
 // every CTA issues back-to-back 128x256 tcgen05.mma instructions on operands that
 // stay in shared memory, so the result is the dense MMA rate of one B200 at the
 // clock it runs at, with no memory traffic. Built as libblprobe.so; bench.py uses it
@@ -93,7 +95,39 @@ __global__ void __launch_bounds__(256) warp_mma_kernel(int iters, int* sink) {
   if (s == 0x7fffffff) sink[threadIdx.x] = s;   // keeps the loop alive
 }
 
+// Failure-detection self-test: one thread waits, with the library's bounded wait, on an
+// mbarrier that nothing ever arrives on. The wait must give up after kWaitTimeoutNs and
+// the kernel must return normally, leaving the context usable; it records the outcome
+// and the time waited.
+__global__ void wait_timeout_kernel(unsigned int* out) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    bl::mbar_init(bl::smem_u32(&bar), 1);
+    abort_flag = 0;
+    bl::fence_mbar_init();
+    const uint64_t t0 = bl::global_timer_ns();
+    const bool got = bl::mbar_wait(bl::smem_u32(&bar), 0, &abort_flag);
+    const uint64_t dt = bl::global_timer_ns() - t0;
+    out[0] = got ? 0u : 1u;
+    out[1] = static_cast<unsigned int>(dt / 1000000ull);
+  }
+}
+
 }  // namespace
+
+// Runs the bounded-wait self-test (about 2 s). out_host[0] = 1 if the wait gave up (the
+// expected outcome), out_host[1] = milliseconds waited. Returns 0, or -1 on a CUDA error.
+extern "C" int blprobe_wait_timeout(unsigned int* out_host, void* stream) {
+  static unsigned int* out = nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!out && cudaMalloc(&out, 2 * sizeof(unsigned int)) != cudaSuccess) return -1;
+  if (cudaMemsetAsync(out, 0, 2 * sizeof(unsigned int), st) != cudaSuccess) return -1;
+  wait_timeout_kernel<<<1, 32, 0, st>>>(out);
+  if (cudaGetLastError() != cudaSuccess) return -1;
+  if (cudaMemcpyAsync(out_host, out, 2 * sizeof(unsigned int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return -1;
+  return cudaStreamSynchronize(st) == cudaSuccess ? 0 : -1;
+}
 
 // Warp-MMA probe: `kind` 2 (s8 m16n8k32) or 3 (b1 m16n8k256); `blocks` x 256 threads,
 // `iters` x 8 MMAs per warp. The caller times it. Returns 0 or -1.

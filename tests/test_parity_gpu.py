@@ -368,3 +368,24 @@ def test_grad_x_int8_dy_training_shape():
     out = B.bitlinear_grad_x_i8(bits_to_dev_bf16(dy), qm["codes"], qm["w_scale"], k_in=k_in)
     torch.cuda.synchronize()
     assert_bf16_within_ulp(bf16_dev_to_bits(out["grad_x"])[rows], y_ref, "grad_x_i8 training shape")
+
+
+# ------------------------------------------------------------------ failure detection
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    # A wait on an mbarrier that nothing arrives on must end by itself (about 2 s), report
+    # it, and leave the context usable: no fault, trap or hang.
+    import ctypes
+    import os
+    probe = ctypes.CDLL(os.path.join(os.path.dirname(B.__file__), "libblprobe.so"))
+    probe.blprobe_wait_timeout.restype = ctypes.c_int
+    probe.blprobe_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    out = (ctypes.c_uint * 2)()
+    assert probe.blprobe_wait_timeout(out, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+    assert out[0] == 1, "the bounded wait did not give up"
+    assert 1500 <= out[1] <= 10000, f"gave up after {out[1]} ms"
+    # the context still runs kernels of the library
+    xq, a = B.bitlinear_act_quant(torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    assert int(xq.abs().sum()) == 0
