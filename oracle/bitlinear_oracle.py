@@ -318,6 +318,63 @@ def grad_x_int8_dy(dy_bits: np.ndarray, mcode: np.ndarray, gamma: np.float32,
     return acc, y, q, a
 
 
+# --------------------------------------------------------------------------- 2:4 storage
+
+def compress_2_4(mcode: np.ndarray, keep: np.ndarray) -> dict:
+    """2:4 structured storage of masked ternary codes (the form sparse tensor cores take).
+
+    Follows: Sparse-BitNet article section 七 (NVIDIA's sparse tensor cores need the 2:4
+    pattern: at most two nonzero weights in every aligned group of four along K).
+    reading: every aligned group of 4 stores exactly two values and their positions
+    i0 < i1 (2 bits each). Kept positions come first in increasing order; a group with
+    fewer than two kept positions is completed with the lowest unused positions, whose
+    stored value is 0. Metadata byte j of a row holds group 2j in bits 0-3 and group
+    2j+1 in bits 4-7, each nibble = i0 | (i1 << 2). Masks with more than two kept
+    positions in a group (6:8, 4:8, 3:8) are not 2:4-valid and raise ValueError.
+    Returns {"values": int8 [rows, K/2], "idx": uint8 [rows, K/4, 2], "meta": uint8 [rows, K/8]}.
+    """
+    c = np.asarray(mcode, dtype=np.int8)
+    kp = np.asarray(keep, dtype=bool)
+    rows, k = c.shape
+    assert k % 8 == 0
+    values = np.zeros((rows, k // 2), dtype=np.int8)
+    idx = np.zeros((rows, k // 4, 2), dtype=np.uint8)
+    meta = np.zeros((rows, k // 8), dtype=np.uint8)
+    for r in range(rows):
+        for g in range(k // 4):
+            kept = [j for j in range(4) if kp[r, 4 * g + j]]
+            if len(kept) > 2:
+                raise ValueError(f"row {r} group {g}: {len(kept)} kept positions, not 2:4-valid")
+            pos = list(kept)
+            for j in range(4):
+                if len(pos) == 2:
+                    break
+                if j not in pos:
+                    pos.append(j)
+            pos.sort()
+            for s_, j in enumerate(pos):
+                values[r, 2 * g + s_] = c[r, 4 * g + j] if kp[r, 4 * g + j] else 0
+                idx[r, g, s_] = j
+            nib = pos[0] | (pos[1] << 2)
+            meta[r, g // 2] |= np.uint8(nib << (4 * (g % 2)))
+    return {"values": values, "idx": idx, "meta": meta}
+
+
+def decompress_2_4(values: np.ndarray, meta: np.ndarray) -> np.ndarray:
+    """Inverse of compress_2_4: scatter each group's two values to the positions its
+    metadata nibble names. Returns int8 [rows, K]."""
+    rows, half = values.shape
+    k = 2 * half
+    out = np.zeros((rows, k), dtype=np.int8)
+    for r in range(rows):
+        for g in range(k // 4):
+            nib = (int(meta[r, g // 2]) >> (4 * (g % 2))) & 0xF
+            i0, i1 = nib & 3, nib >> 2
+            out[r, 4 * g + i0] = values[r, 2 * g]
+            out[r, 4 * g + i1] = values[r, 2 * g + 1]
+    return out
+
+
 # --------------------------------------------------------------------------- diagnostics
 
 HIST_BINS = 17   # [k/8, (k+1)/8) of gamma for k = 0..15, then [2, inf)

@@ -494,3 +494,44 @@ def test_grad_x_int8_dy_error_within_quantisation_bound():
     bound = (np.abs(mcode).sum(axis=0)[None, :] * float(gamma) * a.astype(np.float64)[:, None] / 254.0) * (1 + 1e-6)
     assert np.all(np.abs(y - exact) <= bound)
     assert np.max(np.abs(y - exact)) > 0   # the approximation is not exact in general
+
+
+# ----------------------------------------------------------------------- 2:4 storage
+
+
+def test_hand_compress_2_4():
+    w = _w_example()
+    qm = O.quant_mask(w, 2, 4)
+    sp = O.compress_2_4(qm["mcode"], qm["keep"])
+    assert sp["values"].ravel().tolist() == _ints("sp24_values")
+    assert sp["meta"].ravel().tolist() == _ints("sp24_meta")
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (2, 8), (1, 8)])
+def test_compress_2_4_round_trip_and_valid_metadata(n, m):
+    w = _tied_weights(13, 8, 128)
+    qm = O.quant_mask(w, n, m)
+    sp = O.compress_2_4(qm["mcode"], qm["keep"])
+    assert np.array_equal(O.decompress_2_4(sp["values"], sp["meta"]), qm["mcode"])
+    nibbles = np.concatenate([sp["meta"] & 0xF, sp["meta"] >> 4], axis=1).ravel()
+    assert set(np.unique(nibbles).tolist()) <= {0x4, 0x8, 0xC, 0x9, 0xD, 0xE}   # i0 < i1
+    # the product over the stored form equals the product over the masked codes
+    rng = np.random.default_rng(3)
+    q = rng.integers(-128, 128, size=(5, 128)).astype(np.int8)
+    dense = q.astype(np.int64) @ qm["mcode"].astype(np.int64).T
+    k = 128
+    g = np.arange(k // 4)
+    acc = np.zeros((5, 8), dtype=np.int64)
+    for r in range(8):
+        for gi in g:
+            for s_ in range(2):
+                acc[:, r] += q[:, 4 * gi + sp["idx"][r, gi, s_]].astype(np.int64) * int(sp["values"][r, 2 * gi + s_])
+    assert np.array_equal(acc, dense)
+
+
+@pytest.mark.parametrize("n,m", [(6, 8), (4, 8), (3, 8), (3, 4)])
+def test_compress_2_4_rejects_denser_masks(n, m):
+    w = _tied_weights(14, 4, 64)
+    qm = O.quant_mask(w, n, m)
+    with pytest.raises(ValueError):
+        O.compress_2_4(qm["mcode"], qm["keep"])
