@@ -197,9 +197,11 @@ def bitlinear_grad_x_i8(dy: torch.Tensor, codes: torch.Tensor, w_scale: torch.Te
     _need(dy, torch.bfloat16, None, "dy")
     if k_in is None:
         k_in = codes.shape[1] * 4
+    _need(codes, torch.uint8, (n_out, k_in // 4), "codes")
     dev = dy.device
     if grad_x is None:
         grad_x = torch.empty((t, k_in), dtype=torch.bfloat16, device=dev)
+    _need(grad_x, torch.bfloat16, (t, k_in), "grad_x")
     acc = torch.empty((t, k_in), dtype=torch.int32, device=dev) if want_acc else None
     need = bitlinear_grad_x_i8_workspace_size(t, k_in, n_out)
     if workspace is None and need:
@@ -216,8 +218,13 @@ def bitlinear_mask_threshold_hist(w: torch.Tensor, mask: torch.Tensor, w_scale: 
     (width 1/8, last bin >= 2), dropped weights, dropped weights with a nonzero code."""
     n_out, k_in = w.shape
     _need(w, torch.float32, None, "w")
+    if m_group not in (4, 8):
+        raise ValueError("m_group must be 4 or 8")
+    _need(mask, torch.uint8, (n_out, k_in // m_group), "mask")
+    _need(w_scale, torch.float32, None, "w_scale")
     if out is None:
         out = torch.empty((19,), dtype=torch.int64, device=w.device)
+    _need(out, torch.int64, (19,), "out")
     st = lib().bitlinear_mask_threshold_hist(_ptr(w), _ptr(mask), _ptr(w_scale), n_out, k_in, m_group, _ptr(out),
                                              _stream(stream))
     check(st, "bitlinear_mask_threshold_hist")
