@@ -538,10 +538,23 @@ def _tile_rows(a, n):
 
 def cpu_baseline(tokens: int) -> dict:
     r = oracle_sample(oracle_inputs(tokens, None))
-    return {"value": round(TOKENS / r["step_s"], 2), "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": (f"full mask/ternary recompute of the 3 weight tensors ({r['mask_s']:.2f} s) + {tokens} of "
-                       f"{TOKENS} tokens through act-quant/fwd/grad_x/grad_w ({r['tokens_s']:.2f} s), "
-                       f"step time extrapolated linearly in tokens")}
+    out = {"value": round(TOKENS / r["step_s"], 2), "unit": "tok/s", "cores": _blas_threads(), "kind": "oracle",
+           "sample": (f"full mask/ternary recompute of the 3 weight tensors ({r['mask_s']:.2f} s) + {tokens} of "
+                      f"{TOKENS} tokens through act-quant/fwd/grad_x/grad_w ({r['tokens_s']:.2f} s), "
+                      f"step time extrapolated linearly in tokens")}
+    # the same oracle on one host thread, on a smaller sample
+    try:
+        from threadpoolctl import threadpool_limits
+        st_tokens, st_rows = max(16, tokens // 4), 1024
+        with threadpool_limits(limits=1):
+            r1 = oracle_sample(oracle_inputs(st_tokens, st_rows, seed_off=7))
+        out["single_thread"] = {
+            "value": round(TOKENS / r1["step_s"], 2), "unit": "tok/s", "cores": 1,
+            "sample": (f"first {st_rows} rows of each weight tensor (scaled to all rows) + {st_tokens} tokens, "
+                       f"one BLAS thread")}
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference(args) -> None:
