@@ -77,6 +77,45 @@ def test_hand_act_quant_and_acc():
     assert int(acc[0, 0]) == _ints("acc_6_8")[0]
 
 
+# ----------------------------------------------------------------------- ties and operation order
+
+def test_hand_ternary_ties_round_to_even():
+    """w/gamma exactly +-0.5 gives code 0 (ties to even), one ulp more gives 1, 1.5 clips."""
+    g = np.float32(float(G["tie_gamma"][0]))
+    half = np.float32(g / np.float32(2))                 # exact in fp32
+    assert float(half) * 2 == float(g)
+    w = np.array([half, -half, np.nextafter(half, np.float32(1)), np.float32(1.5) * g], dtype=np.float32)
+    assert float(w[3] / g) == 1.5                        # the last ratio is exactly 1.5 as well
+    assert O.ternary_codes(w, g).tolist() == _ints("tie_codes")
+
+
+def _bf16_row(key):
+    vals = np.array([float(t) for t in G[key]], dtype=np.float32)
+    bits = synth.f32_to_bf16_bits(vals)
+    assert np.array_equal(O.bf16_to_f32(bits), vals), "every value of the row is a bf16"
+    return bits.reshape(1, -1)
+
+
+def test_hand_act_quant_ties_round_to_even():
+    q, a = O.act_quant(_bf16_row("tie_x"))
+    assert float(a[0]) == 127.0
+    assert q.ravel().tolist() == _ints("tie_q")
+
+
+def test_hand_act_quant_scale_then_one_multiply():
+    """Row B of the golden file: s = fp32(127/a) first, then one fp32 multiply. The other
+    operation orders (x*127 first, or exact arithmetic) give 64 instead of 63."""
+    row = _bf16_row("order_x")
+    q, a = O.act_quant(row)
+    assert float(a[0]) == 1.1875
+    assert q.ravel().tolist() == _ints("order_q")
+    # the worked intermediate values, exactly as rationals
+    s = np.float32(np.float32(127) / np.float32(1.1875))
+    assert Fraction(float(s)) == Fraction(14017805, 2 ** 17)
+    assert Fraction(float(np.float32(np.float32(0.59375) * s))) == Fraction(16646143, 2 ** 18)
+    assert Fraction(0.59375) * 127 / Fraction(1.1875) == Fraction(127, 2)
+
+
 # ----------------------------------------------------------------------- gamma: exact rationals
 
 def _exact_mean(w):
