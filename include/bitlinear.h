@@ -107,7 +107,10 @@ bl_status bitlinear_quant_mask_status(const void* workspace, void* stream);
  * GPU that loads the library holds it until exit), which limits the tensor to
  * n_out * k_in <= 4966055936 weights; larger tensors get BL_ERR_UNSUPPORTED_SHAPE.
  * The first call on each device looks up that array's device address (with the
- * device current); make that first call before any stream capture. All calls on a
+ * device current) and keeps it for the life of the process; make that first call
+ * before any stream capture. A reset of the device's primary context
+ * (cudaDeviceReset) invalidates the kept address: do not call this entry point on a
+ * device after resetting it. All calls on a
  * device share the array, so calls that overlap on the GPU race: order them on one
  * stream. A range error shows as gamma = NaN and all-zero codes (there is no
  * workspace to read a status from).
@@ -139,6 +142,10 @@ bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t
  *   w_scale [1] fp32 gamma. acc_out [t, n_out] int32, out, nullable.
  *   y_out [t, n_out], out, bf16 (y_dtype = BL_OUT_BF16) or fp32 (BL_OUT_F32).
  * No bias term.
+ * The kernel for up to 8 tokens from codes keeps a lookup table at a fixed shared-memory
+ * address: its first use on each device runs a one-CTA check of the shared-memory layout
+ * and synchronises `stream` (make that first call before any stream capture). Where the
+ * table does not fit, every such call returns BL_ERR_CUDA before enqueueing anything.
  */
 bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* codes, const int8_t* w_i8,
                         const float* w_scale, int64_t t, int64_t k_in, int64_t n_out, int32_t* acc_out, void* y_out,
@@ -163,28 +170,47 @@ typedef struct {
  * packed 2-bit codes are streamed once per 128 tokens (once per 8 tokens when the
  * largest problem has at most 8). `problems` is a HOST array
  * (copied into the launch); y_dtype applies to all problems. Problems may have t = 0.
+ * The one-time layout check of bitlinear_fwd applies here too (batches of up to 8).
  * More than 256 problems: BL_ERR_UNSUPPORTED_SHAPE.
  */
 bl_status bitlinear_fwd_grouped(const bl_fwd_problem* problems, int count, int y_dtype, void* stream);
 
-/* Bytes of workspace bitlinear_bwd needs (0 when grad_x is not requested). */
-size_t bitlinear_bwd_workspace_size(int64_t t, int64_t k_in, int64_t n_out, int want_grad_x);
+/* Flags of bitlinear_bwd. */
+enum {
+  /* grad_w against the activations the forward product consumed, q * a_t / 127
+   * (from bitlinear_act_quant), instead of the layer's bf16 input x. */
+  BL_GRADW_DEQUANT_X = 1
+};
+
+/* Bytes of workspace bitlinear_bwd needs (0 when neither grad_x nor the
+ * BL_GRADW_DEQUANT_X option is requested). */
+size_t bitlinear_bwd_workspace_size(int64_t t, int64_t k_in, int64_t n_out, int want_grad_x, int flags);
 
 /*
- * Steps a5 + a6: the dual straight-through backward.
+ * Steps a5 + a6: the dual straight-through backward (Sparse-BitNet article, section
+ * 三: masked weights still receive gradients; section 六: the estimator passes the
+ * gradient through both the quantiser and the mask).
  *   grad_x[t, k] = sum_n dy[t, n] * gamma * masked_code[n, k]   (bf16 out, fp32 accumulate)
- *   grad_w[n, k] = sum_t dy[t, n] * x[t, k]   for EVERY latent weight, masked ones
+ *   grad_w[n, k] = sum_t dy[t, n] * X[t, k]   for EVERY latent weight, masked ones
  *                  included (the mask does not enter; fp32 accumulate).
+ *   X is the layer's bf16 input x by default. With flags & BL_GRADW_DEQUANT_X it is
+ *   the dequantised int8 input, X[t, k] = bf16(q[t, k] * fp32(a_t / 127)): what the
+ *   forward product consumed. The pages say only "straight-through"; both readings
+ *   are offered.
  *
- *   dy [t, n_out] bf16, x [t, k_in] bf16 (the layer's bf16 input).
+ *   dy [t, n_out] bf16. x [t, k_in] bf16 (needed for grad_w without the flag).
+ *   xq [t, k_in] int8 and absmax [t] fp32 (needed for grad_w with the flag).
  *   codes [n_out, k_in / 4] packed masked codes, w_scale [1] gamma (needed for grad_x).
  *   grad_x [t, k_in] bf16, out, nullable. grad_w [n_out, k_in], out, nullable, bf16
  *   (grad_w_dtype = BL_OUT_BF16) or fp32 (BL_OUT_F32). With t = 0, grad_w is zeroed.
- *   workspace bitlinear_bwd_workspace_size() bytes (holds the bf16 ternary matrix).
+ *   flags: 0 or BL_GRADW_DEQUANT_X (other bits: BL_ERR_INVALID_ARG).
+ *   workspace bitlinear_bwd_workspace_size() bytes: the bf16 ternary matrix
+ *   [n_out, k_in] (for grad_x) followed by the bf16 X_deq [t, k_in] (with the flag).
  */
-bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* codes, const float* w_scale, int64_t t,
-                        int64_t k_in, int64_t n_out, uint16_t* grad_x, void* grad_w, int grad_w_dtype,
-                        void* workspace, size_t workspace_bytes, void* stream);
+bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const int8_t* xq, const float* absmax,
+                        const uint8_t* codes, const float* w_scale, int64_t t, int64_t k_in, int64_t n_out,
+                        uint16_t* grad_x, void* grad_w, int grad_w_dtype, int flags, void* workspace,
+                        size_t workspace_bytes, void* stream);
 
 /* Bytes of workspace bitlinear_grad_x_i8 needs (0 for an empty problem). */
 size_t bitlinear_grad_x_i8_workspace_size(int64_t t, int64_t k_in, int64_t n_out);
@@ -241,7 +267,7 @@ bl_status bitlinear_device_status(unsigned int* bits);
 /* Message for the calling thread's last non-OK status ("" if none). */
 const char* bitlinear_last_error(void);
 
-/* ABI version of this header: 1. */
+/* ABI version of this header: 2. */
 int bitlinear_abi_version(void);
 
 #ifdef __cplusplus

@@ -43,8 +43,8 @@ SIGNATURES = {
     "bitlinear_act_quant": (_INT, [_P, _I64, _I64, _P, _P, _P]),
     "bitlinear_fwd": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P]),
     "bitlinear_fwd_grouped": (_INT, [_c.POINTER(BlFwdProblem), _INT, _INT, _P]),
-    "bitlinear_bwd_workspace_size": (_SZ, [_I64, _I64, _I64, _INT]),
-    "bitlinear_bwd": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _SZ, _P]),
+    "bitlinear_bwd_workspace_size": (_SZ, [_I64, _I64, _I64, _INT, _INT]),
+    "bitlinear_bwd": (_INT, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _INT, _P, _SZ, _P]),
     "bitlinear_grad_x_i8_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_grad_x_i8": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "bitlinear_mask_threshold_hist": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),

@@ -24,16 +24,44 @@ def _ptr(t) -> int | None:
     return None if t is None else int(t.data_ptr())
 
 
-def _need(t, dtype, shape, name):
+def _need(t, dtype, shape, name, device=None):
+    """Check one caller buffer before its pointer goes to the library (the C ABI
+    cannot see buffer sizes, so an undersized or mistyped buffer must stop here)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError(f"{name}: must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
     if not t.is_contiguous():
         raise ValueError(f"{name}: must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
     return t
+
+
+def _need_vec(t, dtype, min_numel, name, device=None):
+    """A contiguous buffer of at least ``min_numel`` elements (per-token or scalar data)."""
+    _need(t, dtype, None, name, device)
+    if t.numel() < min_numel:
+        raise ValueError(f"{name}: needs at least {min_numel} elements, got {t.numel()}")
+    return t
+
+
+def _need_bytes(t, nbytes, name, device=None):
+    """A contiguous uint8 workspace of at least ``nbytes`` bytes."""
+    return _need_vec(t, torch.uint8, nbytes, name, device)
+
+
+def _check_qm_outputs(o: dict, n_out: int, k_in: int, m_group: int, dev) -> None:
+    _need(o["codes"], torch.uint8, (n_out, k_in // 4), "codes", dev)
+    _need_vec(o["w_scale"], torch.float32, 1, "w_scale", dev)
+    if o.get("mask") is not None:
+        _need(o["mask"], torch.uint8, (n_out, k_in // m_group), "mask", dev)
+    if o.get("w_i8") is not None:
+        _need(o["w_i8"], torch.int8, (n_out, k_in), "w_i8", dev)
 
 
 def bitlinear_quant_mask_workspace_size(n_out: int, k_in: int) -> int:
@@ -60,9 +88,13 @@ def bitlinear_quant_mask(w: torch.Tensor, n_keep: int, m_group: int, *, want_mas
         o["mask"] = torch.empty((n_out, k_in // m_group), dtype=torch.uint8, device=dev)
     if want_w_i8 and "w_i8" not in o:
         o["w_i8"] = torch.empty((n_out, k_in), dtype=torch.int8, device=dev)
+    if m_group not in (4, 8) or k_in % m_group:
+        raise ValueError(f"m_group must be 4 or 8 and divide k_in (got {m_group})")
+    _check_qm_outputs(o, n_out, k_in, m_group, dev)
     ws_bytes = bitlinear_quant_mask_workspace_size(n_out, k_in)
     if workspace is None:
         workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    _need_bytes(workspace, ws_bytes, "workspace", dev)
     st = lib().bitlinear_quant_mask(_ptr(w), n_out, k_in, n_keep, m_group, _ptr(o.get("mask")), _ptr(o["codes"]),
                                     _ptr(o.get("w_i8")), _ptr(o["w_scale"]), _ptr(workspace), workspace.numel(),
                                     _stream(stream))
@@ -86,6 +118,9 @@ def bitlinear_quant_mask_noalloc(w: torch.Tensor, n_keep: int, m_group: int, *, 
     """
     n_out, k_in = w.shape
     _need(w, torch.float32, None, "w")
+    if m_group not in (4, 8) or k_in % m_group:
+        raise ValueError(f"m_group must be 4 or 8 and divide k_in (got {m_group})")
+    _check_qm_outputs(out, n_out, k_in, m_group, w.device)
     st = lib().bitlinear_quant_mask_noalloc(_ptr(w), n_out, k_in, n_keep, m_group, _ptr(out.get("mask")),
                                             _ptr(out["codes"]), _ptr(out.get("w_i8")), _ptr(out["w_scale"]),
                                             _stream(stream))
@@ -102,7 +137,8 @@ def bitlinear_act_quant(x: torch.Tensor, *, xq: torch.Tensor | None = None, absm
         xq = torch.empty((t, k_in), dtype=torch.int8, device=x.device)
     if absmax is None:
         absmax = torch.empty((max(t, 1) + 3) // 4 * 4, dtype=torch.float32, device=x.device)[:t]
-    _need(xq, torch.int8, (t, k_in), "xq")
+    _need(xq, torch.int8, (t, k_in), "xq", x.device)
+    _need_vec(absmax, torch.float32, t, "absmax", x.device)
     st = lib().bitlinear_act_quant(_ptr(x), t, k_in, _ptr(xq), _ptr(absmax), _stream(stream))
     check(st, "bitlinear_act_quant")
     return xq, absmax
@@ -114,12 +150,27 @@ def bitlinear_fwd(xq: torch.Tensor, absmax: torch.Tensor, w_scale: torch.Tensor,
                   stream=None) -> tuple[torch.Tensor, torch.Tensor | None]:
     """y = (xq . masked_codes^T) * absmax/127 * gamma; returns (y, acc or None)."""
     t, k_in = xq.shape
+    dev = xq.device
+    _need(xq, torch.int8, None, "xq")
+    if w_i8 is None and codes is None:
+        raise ValueError("give codes or w_i8")
     if n_out is None:
         n_out = (w_i8 if w_i8 is not None else codes).shape[0]
+    if codes is not None:
+        _need(codes, torch.uint8, (n_out, k_in // 4), "codes", dev)
+    if w_i8 is not None:
+        _need(w_i8, torch.int8, (n_out, k_in), "w_i8", dev)
+    _need_vec(absmax, torch.float32, t, "absmax", dev)
+    _need_vec(w_scale, torch.float32, 1, "w_scale", dev)
     if y is None:
-        y = torch.empty((t, n_out), dtype=y_dtype, device=xq.device)
+        y = torch.empty((t, n_out), dtype=y_dtype, device=dev)
+    if y.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError(f"y: expected bfloat16 or float32, got {y.dtype}")
+    _need(y, y.dtype, (t, n_out), "y", dev)
     if want_acc and acc is None:
-        acc = torch.empty((t, n_out), dtype=torch.int32, device=xq.device)
+        acc = torch.empty((t, n_out), dtype=torch.int32, device=dev)
+    if acc is not None:
+        _need(acc, torch.int32, (t, n_out), "acc", dev)
     ydt = BL_OUT_F32 if y.dtype == torch.float32 else BL_OUT_BF16
     st = lib().bitlinear_fwd(_ptr(xq), _ptr(absmax), _ptr(codes), _ptr(w_i8), _ptr(w_scale), t, k_in, n_out,
                              _ptr(acc), _ptr(y), ydt, _stream(stream))
@@ -138,14 +189,22 @@ def bitlinear_fwd_grouped(problems: list[dict], *, y_dtype=torch.bfloat16, strea
     out = []
     for i, p in enumerate(problems):
         xq, codes = p["xq"], p["codes"]
+        _need(xq, torch.int8, None, f"problem {i} xq")
         t, k_in = xq.shape
+        dev = xq.device
         n_out = codes.shape[0]
+        _need(codes, torch.uint8, (n_out, k_in // 4), f"problem {i} codes", dev)
+        _need_vec(p["absmax"], torch.float32, t, f"problem {i} absmax", dev)
+        _need_vec(p["w_scale"], torch.float32, 1, f"problem {i} w_scale", dev)
         y = p.get("y")
         if y is None:
-            y = torch.empty((t, n_out), dtype=y_dtype, device=xq.device)
+            y = torch.empty((t, n_out), dtype=y_dtype, device=dev)
+        _need(y, y_dtype, (t, n_out), f"problem {i} y", dev)
         acc = p.get("acc")
         if acc is None and p.get("want_acc"):
-            acc = torch.empty((t, n_out), dtype=torch.int32, device=xq.device)
+            acc = torch.empty((t, n_out), dtype=torch.int32, device=dev)
+        if acc is not None:
+            _need(acc, torch.int32, (t, n_out), f"problem {i} acc", dev)
         arr[i] = _lib.BlFwdProblem(_ptr(xq), _ptr(p["absmax"]), _ptr(codes), _ptr(p["w_scale"]), t, k_in, n_out,
                                    _ptr(acc), _ptr(y))
         out.append({**p, "y": y, "acc": acc})
@@ -155,31 +214,63 @@ def bitlinear_fwd_grouped(problems: list[dict], *, y_dtype=torch.bfloat16, strea
     return out
 
 
-def bitlinear_bwd_workspace_size(t: int, k_in: int, n_out: int, want_grad_x: bool = True) -> int:
-    return int(lib().bitlinear_bwd_workspace_size(t, k_in, n_out, int(want_grad_x)))
+BL_GRADW_DEQUANT_X = 1   # grad_W against the dequantised activations q * a / 127
+
+
+def bitlinear_bwd_workspace_size(t: int, k_in: int, n_out: int, want_grad_x: bool = True, flags: int = 0) -> int:
+    return int(lib().bitlinear_bwd_workspace_size(t, k_in, n_out, int(want_grad_x), int(flags)))
 
 
 def bitlinear_bwd(dy: torch.Tensor, x: torch.Tensor | None, codes: torch.Tensor | None, w_scale: torch.Tensor | None, *,
                   want_grad_x: bool = True, want_grad_w: bool = True, grad_w_dtype=torch.bfloat16,
                   grad_x: torch.Tensor | None = None, grad_w: torch.Tensor | None = None,
                   workspace: torch.Tensor | None = None, k_in: int | None = None,
+                  xq: torch.Tensor | None = None, absmax: torch.Tensor | None = None, flags: int = 0,
                   stream=None) -> tuple[torch.Tensor | None, torch.Tensor | None]:
-    """Dual straight-through backward; returns (grad_x or None, grad_w or None)."""
+    """Dual straight-through backward; returns (grad_x or None, grad_w or None).
+
+    ``flags = BL_GRADW_DEQUANT_X`` computes grad_w against q * a / 127 (``xq`` and
+    ``absmax`` from bitlinear_act_quant) instead of the bf16 input ``x``.
+    """
     t, n_out = dy.shape
     _need(dy, torch.bfloat16, None, "dy")
-    if k_in is None:
-        k_in = x.shape[1] if x is not None else codes.shape[1] * 4
     dev = dy.device
+    deq = bool(flags & BL_GRADW_DEQUANT_X)
+    if k_in is None:
+        k_in = (xq.shape[1] if deq and xq is not None else
+                x.shape[1] if x is not None else codes.shape[1] * 4)
     if want_grad_x and grad_x is None:
         grad_x = torch.empty((t, k_in), dtype=torch.bfloat16, device=dev)
     if want_grad_w and grad_w is None:
         grad_w = torch.empty((n_out, k_in), dtype=grad_w_dtype, device=dev)
+    if grad_x is not None:
+        _need(grad_x, torch.bfloat16, (t, k_in), "grad_x", dev)
+        if codes is None or w_scale is None:
+            raise ValueError("grad_x needs codes and w_scale")
+    if codes is not None:
+        _need(codes, torch.uint8, (n_out, k_in // 4), "codes", dev)
+    if w_scale is not None:
+        _need_vec(w_scale, torch.float32, 1, "w_scale", dev)
+    if grad_w is not None:
+        if grad_w.dtype not in (torch.bfloat16, torch.float32):
+            raise TypeError(f"grad_w: expected bfloat16 or float32, got {grad_w.dtype}")
+        _need(grad_w, grad_w.dtype, (n_out, k_in), "grad_w", dev)
+        if deq:
+            if xq is None or absmax is None:
+                raise ValueError("BL_GRADW_DEQUANT_X needs xq and absmax")
+            _need(xq, torch.int8, (t, k_in), "xq", dev)
+            _need_vec(absmax, torch.float32, t, "absmax", dev)
+        elif x is not None:
+            _need(x, torch.bfloat16, (t, k_in), "x", dev)
     gwdt = BL_OUT_F32 if (grad_w is not None and grad_w.dtype == torch.float32) else BL_OUT_BF16
-    need = bitlinear_bwd_workspace_size(t, k_in, n_out, grad_x is not None)
+    need = bitlinear_bwd_workspace_size(t, k_in, n_out, grad_x is not None, flags if grad_w is not None else 0)
     if need and workspace is None:
         workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
-    st = lib().bitlinear_bwd(_ptr(dy), _ptr(x), _ptr(codes), _ptr(w_scale), t, k_in, n_out, _ptr(grad_x), _ptr(grad_w),
-                             gwdt, _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
+    if workspace is not None:
+        _need_bytes(workspace, need, "workspace", dev)
+    st = lib().bitlinear_bwd(_ptr(dy), _ptr(x), _ptr(xq), _ptr(absmax), _ptr(codes), _ptr(w_scale), t, k_in, n_out,
+                             _ptr(grad_x), _ptr(grad_w), gwdt, int(flags), _ptr(workspace),
+                             0 if workspace is None else workspace.numel(), _stream(stream))
     check(st, "bitlinear_bwd")
     return grad_x, grad_w
 
@@ -203,9 +294,12 @@ def bitlinear_grad_x_i8(dy: torch.Tensor, codes: torch.Tensor, w_scale: torch.Te
         grad_x = torch.empty((t, k_in), dtype=torch.bfloat16, device=dev)
     _need(grad_x, torch.bfloat16, (t, k_in), "grad_x")
     acc = torch.empty((t, k_in), dtype=torch.int32, device=dev) if want_acc else None
+    _need_vec(w_scale, torch.float32, 1, "w_scale", dev)
     need = bitlinear_grad_x_i8_workspace_size(t, k_in, n_out)
     if workspace is None and need:
         workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    if workspace is not None:
+        _need_bytes(workspace, need, "workspace", dev)
     st = lib().bitlinear_grad_x_i8(_ptr(dy), _ptr(codes), _ptr(w_scale), t, k_in, n_out, _ptr(grad_x), _ptr(acc),
                                    _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
     check(st, "bitlinear_grad_x_i8")
@@ -220,11 +314,11 @@ def bitlinear_mask_threshold_hist(w: torch.Tensor, mask: torch.Tensor, w_scale: 
     _need(w, torch.float32, None, "w")
     if m_group not in (4, 8):
         raise ValueError("m_group must be 4 or 8")
-    _need(mask, torch.uint8, (n_out, k_in // m_group), "mask")
-    _need(w_scale, torch.float32, None, "w_scale")
+    _need(mask, torch.uint8, (n_out, k_in // m_group), "mask", w.device)
+    _need_vec(w_scale, torch.float32, 1, "w_scale", w.device)
     if out is None:
         out = torch.empty((19,), dtype=torch.int64, device=w.device)
-    _need(out, torch.int64, (19,), "out")
+    _need(out, torch.int64, (19,), "out", w.device)
     st = lib().bitlinear_mask_threshold_hist(_ptr(w), _ptr(mask), _ptr(w_scale), n_out, k_in, m_group, _ptr(out),
                                              _stream(stream))
     check(st, "bitlinear_mask_threshold_hist")
@@ -247,5 +341,5 @@ __all__ = [
     "bitlinear_quant_mask_noalloc",
     "bitlinear_act_quant", "bitlinear_fwd", "bitlinear_fwd_grouped", "bitlinear_bwd_workspace_size", "bitlinear_bwd",
     "bitlinear_grad_x_i8_workspace_size", "bitlinear_grad_x_i8", "bitlinear_mask_threshold_hist",
-    "bitlinear_device_status", "bitlinear_abi_version", "BL_OUT_BF16", "BL_OUT_F32", "_lib",
+    "bitlinear_device_status", "bitlinear_abi_version", "BL_OUT_BF16", "BL_OUT_F32", "BL_GRADW_DEQUANT_X", "_lib",
 ]

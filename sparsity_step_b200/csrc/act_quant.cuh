@@ -161,3 +161,35 @@ __global__ void __launch_bounds__(256) act_quant_long_kernel(const uint4* __rest
 }
 
 }  // namespace bl
+
+namespace bl {
+
+// Dequantised activations for the optional grad_W reading: x_deq[t, k] = q[t, k] * a_t / 127
+// rounded to bf16 (one fp32 division per row, one fp32 multiply per element, then
+// round to nearest even). One thread = 16 int8 elements of one row (k_in % 64 == 0,
+// so a 16-element chunk never crosses a row): one 16-byte load, two 16-byte stores.
+__global__ void __launch_bounds__(256) dequant_x_bf16_kernel(const uint4* __restrict__ xq, const float* __restrict__ absmax,
+                                                             int64_t nchunks, int k16, uint4* __restrict__ out) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nchunks; i += stride) {
+    const float sc = __fdiv_rn(absmax[i / k16], 127.0f);
+    const uint4 v = xq[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t b = w[j] >> (16 * h);
+        const float f0 = __fmul_rn(static_cast<float>(static_cast<int8_t>(b & 0xffu)), sc);
+        const float f1 = __fmul_rn(static_cast<float>(static_cast<int8_t>((b >> 8) & 0xffu)), sc);
+        const __nv_bfloat162 p = __floats2bfloat162_rn(f0, f1);
+        o[2 * j + h] = *reinterpret_cast<const uint32_t*>(&p);
+      }
+    }
+    out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+}  // namespace bl

@@ -157,16 +157,62 @@ inline bool use_cta_pair(int64_t m) { return m > bl::kBM; }
 
 // ------------------------------------------------------------------ grouped codes product
 
+// The warp-MMA decode kernel keeps its lookup table at a fixed shared-window address
+// (bl::kDecLutAddr) below which its first ring slot must fit. Where the dynamic shared
+// memory starts depends on the device and the driver, so the first launch on each device
+// runs one CTA of the kernel in probe mode, reads that address back (synchronously: the
+// first call must not be under stream capture) and remembers the verdict. A device
+// where the table does not fit gets BL_ERR_CUDA from every call, before anything is
+// enqueued, instead of a launch that would leave y unwritten.
+constexpr int kMaxLayoutDevices = 64;
+int g_dec_layout[kMaxLayoutDevices] = {};   // 0 unchecked, 1 fits, -1 does not fit
+unsigned int g_dec_base_seen[kMaxLayoutDevices] = {};
+std::mutex g_dec_layout_mu;
+
+template <int NG>
+bl_status check_decode_layout(cudaStream_t st) {
+  using C = bl::DecCfg<NG>;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxLayoutDevices) return fail(BL_ERR_INVALID_ARG, "device ordinal %d not supported", dev);
+  std::lock_guard<std::mutex> lock(g_dec_layout_mu);
+  if (g_dec_layout[dev] == 0) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(st, &cap);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    if (cap != cudaStreamCaptureStatusNone)
+      return fail(BL_ERR_CUDA, "the first decode-kernel call on a device checks its shared-memory layout "
+                               "synchronously: make it before stream capture");
+    e = cudaFuncSetAttribute(bl::fwd_codes_mma_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+    static thread_local bl::FwdGroup probe;   // ~16 KB: kept off the stack
+    probe.count = 0;
+    probe.total_tasks = 0;
+    probe.y_f32 = 0;
+    probe.layout_probe = 1;
+    bl::fwd_codes_mma_kernel<NG><<<1, C::kThreads, C::kSmemBytes, st>>>(probe);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "decode layout probe launch");
+    e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "decode layout probe");
+    unsigned int base = 0;
+    e = cudaMemcpyFromSymbol(&base, bl::g_dec_smem_base, sizeof(base));
+    if (e != cudaSuccess) return cuda_fail(e, "decode layout read");
+    g_dec_base_seen[dev] = base;
+    g_dec_layout[dev] = (base + C::kSlotBytes <= bl::kDecLutAddr) ? 1 : -1;
+  }
+  if (g_dec_layout[dev] < 0)
+    return fail(BL_ERR_CUDA, "decode kernel: dynamic shared memory starts at 0x%x, where its fixed-address lookup "
+                             "table does not fit; use the int8-weight product (w_i8) or batches of 9+ tokens",
+                g_dec_base_seen[dev]);
+  return BL_OK;
+}
+
 template <int NG>
 bl_status launch_fwd_codes_ng(const bl::FwdGroup& grp, cudaStream_t st) {
   using C = bl::DecCfg<NG>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(bl::fwd_codes_mma_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
-    attr_set = true;
-  }
+  if (bl_status s = check_decode_layout<NG>(st)) return s;
   int64_t blocks = (static_cast<int64_t>(grp.total_tasks) + C::kWarps - 1) / C::kWarps;
   const int64_t cap = int64_t(device_sm_count());   // one CTA per SM (persistent)
   if (blocks > cap) blocks = cap;
@@ -204,6 +250,7 @@ bl_status launch_fwd_codes_tc(const bl_fwd_problem* problems, int count, bool y_
   grp.count = n;
   grp.total_tasks = static_cast<int>(tasks);
   grp.y_f32 = y_f32 ? 1 : 0;
+  grp.layout_probe = 0;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(bl::fwd_codes_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -253,6 +300,7 @@ bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32
   grp.count = n;
   grp.total_tasks = static_cast<int>(tasks);
   grp.y_f32 = y_f32 ? 1 : 0;
+  grp.layout_probe = 0;
   return launch_fwd_codes_ng<ng>(grp, st);
 }
 
@@ -389,7 +437,7 @@ inline size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
 
 extern "C" {
 
-int bitlinear_abi_version(void) { return 1; }
+int bitlinear_abi_version(void) { return 2; }
 
 const char* bitlinear_last_error(void) { return g_err; }
 
@@ -477,27 +525,34 @@ bl_status bitlinear_fwd_grouped(const bl_fwd_problem* problems, int count, int y
   return launch_fwd_codes(problems, count, y_dtype == BL_OUT_F32, as_stream(stream));
 }
 
-size_t bitlinear_bwd_workspace_size(int64_t t, int64_t k_in, int64_t n_out, int want_grad_x) {
-  (void)t;
-  if (!want_grad_x || k_in <= 0 || n_out <= 0) return 0;
-  return static_cast<size_t>(n_out) * static_cast<size_t>(k_in) * 2;
+size_t bitlinear_bwd_workspace_size(int64_t t, int64_t k_in, int64_t n_out, int want_grad_x, int flags) {
+  if (k_in <= 0 || n_out <= 0 || t < 0) return 0;
+  size_t b = want_grad_x ? round256(static_cast<size_t>(n_out) * static_cast<size_t>(k_in) * 2) : 0;
+  if (flags & BL_GRADW_DEQUANT_X) b += static_cast<size_t>(t) * static_cast<size_t>(k_in) * 2;
+  return b;
 }
 
-bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* codes, const float* w_scale, int64_t t,
-                        int64_t k_in, int64_t n_out, uint16_t* grad_x, void* grad_w, int grad_w_dtype, void* workspace,
+bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const int8_t* xq, const float* absmax,
+                        const uint8_t* codes, const float* w_scale, int64_t t, int64_t k_in, int64_t n_out,
+                        uint16_t* grad_x, void* grad_w, int grad_w_dtype, int flags, void* workspace,
                         size_t workspace_bytes, void* stream) {
   g_err[0] = 0;
   if (!grad_x && !grad_w) return fail(BL_ERR_INVALID_ARG, "request grad_x, grad_w or both");
+  if (flags & ~BL_GRADW_DEQUANT_X) return fail(BL_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const bool deq = grad_w && (flags & BL_GRADW_DEQUANT_X);
   if (!dy && t != 0) return fail(BL_ERR_INVALID_ARG, "dy is required");
   if (grad_x && (!codes || !w_scale)) return fail(BL_ERR_INVALID_ARG, "grad_x needs codes and w_scale");
-  if (grad_w && !x && t != 0) return fail(BL_ERR_INVALID_ARG, "grad_w needs x");
+  if (grad_w && !deq && !x && t != 0) return fail(BL_ERR_INVALID_ARG, "grad_w needs x");
+  if (deq && (!xq || !absmax) && t != 0)
+    return fail(BL_ERR_INVALID_ARG, "BL_GRADW_DEQUANT_X needs xq and absmax");
   if (grad_w && grad_w_dtype != BL_OUT_BF16 && grad_w_dtype != BL_OUT_F32)
     return fail(BL_ERR_INVALID_ARG, "grad_w_dtype must be BL_OUT_BF16 or BL_OUT_F32");
   if (bl_status s = check_shape(t, k_in, n_out)) return s;
-  if ((dy && !aligned16(dy)) || (x && !aligned16(x)) || (codes && !aligned16(codes)) || (w_scale && !aligned16(w_scale)) ||
-      (grad_x && !aligned16(grad_x)) || (grad_w && !aligned16(grad_w)) || (workspace && !aligned16(workspace)))
+  if ((dy && !aligned16(dy)) || (x && !aligned16(x)) || (xq && !aligned16(xq)) || (absmax && !aligned16(absmax)) ||
+      (codes && !aligned16(codes)) || (w_scale && !aligned16(w_scale)) || (grad_x && !aligned16(grad_x)) ||
+      (grad_w && !aligned16(grad_w)) || (workspace && !aligned16(workspace)))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
-  const size_t need = bitlinear_bwd_workspace_size(t, k_in, n_out, grad_x != nullptr);
+  const size_t need = bitlinear_bwd_workspace_size(t, k_in, n_out, grad_x != nullptr, deq ? BL_GRADW_DEQUANT_X : 0);
   if (need && (!workspace || workspace_bytes < need))
     return fail(BL_ERR_WORKSPACE, "workspace too small: %zu < %zu", workspace_bytes, need);
   cudaStream_t st = as_stream(stream);
@@ -544,10 +599,24 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const uint8_t* co
       if (bl_status s = launch_gemm<false, false, true, bl::EPI_GRADX, true>(ta, tb, to, g, st)) return s;
   }
   if (grad_w) {
+    const void* xb = x;
+    if (deq) {   // X_deq = q * a / 127 in bf16, after the ternary matrix in the workspace
+      uint8_t* xd = static_cast<uint8_t*>(workspace) +
+                    (grad_x ? round256(static_cast<size_t>(n_out) * static_cast<size_t>(k_in) * 2) : 0);
+      const int64_t nchunks = t * k_in / 16;
+      int64_t grid = (nchunks + 255) / 256;
+      const int64_t cap = int64_t(device_sm_count()) * 16;
+      if (grid > cap) grid = cap;
+      bl::dequant_x_bf16_kernel<<<(int)grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(xq), absmax, nchunks,
+                                                          static_cast<int>(k_in / 16), reinterpret_cast<uint4*>(xd));
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+      xb = xd;
+    }
     CUtensorMap ta, tb;
     // A = dY^T: dY [t, n_out] read MN-major (reduction over t); B = X [t, k_in], MN-major
     if (bl_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dy, n_out, t, 64, 64)) return s;
-    if (bl_status s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, k_in, t, 64, 64)) return s;
+    if (bl_status s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, xb, k_in, t, 64, 64)) return s;
     bl::GemmArgs g{};
     g.M = static_cast<int>(n_out);
     g.N = static_cast<int>(k_in);

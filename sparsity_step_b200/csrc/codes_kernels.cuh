@@ -74,7 +74,12 @@ struct FwdGroup {
   int count;
   int total_tasks;
   int y_f32;
+  int layout_probe;   // fwd_codes_mma_kernel: record where dynamic shared memory starts, do nothing else
 };
+
+// Shared-window address of fwd_codes_mma_kernel's dynamic shared memory, written by a
+// one-CTA launch with layout_probe set (the host checks it once per device).
+__device__ unsigned int g_dec_smem_base;
 
 __device__ __forceinline__ void mma_m16n8k32_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                 uint32_t b0, uint32_t b1) {
@@ -241,6 +246,10 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
   using C = DecCfg<NG>;
   extern __shared__ __align__(1024) uint8_t dsmem[];
   const uint32_t base = smem_u32(dsmem);
+  if (G.layout_probe) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) g_dec_smem_base = base;
+    return;
+  }
   if (base + C::kSlotBytes > kDecLutAddr) {   // slot 0 would overlap the table: do nothing
     if (threadIdx.x == 0) atomicOr(&g_device_status, DEV_ST_SMEM_LAYOUT);
     return;

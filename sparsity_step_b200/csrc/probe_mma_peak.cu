@@ -67,34 +67,6 @@ __global__ void __launch_bounds__(kProbeThreads, 1) mma_peak_kernel(int iters, u
   }
 }
 
-// Legacy warp-level MMA probes (independent accumulators, operands in registers):
-// kind 2 = m16n8k32 s8 (mma.sync), kind 3 = m16n8k256 b1 and.popc.
-template <int KIND>
-__global__ void __launch_bounds__(256) warp_mma_kernel(int iters, int* sink) {
-  int acc[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0;
-  uint32_t a0 = threadIdx.x * 0x01010101u, a1 = a0 ^ 0x5A5A5A5Au, a2 = a0 + 7u, a3 = a1 * 3u;
-  uint32_t b0 = a0 ^ 0x33333333u, b1 = a1 ^ 0x0F0F0F0Fu;
-  for (int it = 0; it < iters; ++it) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (KIND == 2)
-        asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-                     : "+r"(acc[i][0]), "+r"(acc[i][1]), "+r"(acc[i][2]), "+r"(acc[i][3])
-                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-      else
-        asm volatile("mma.sync.aligned.m16n8k256.row.col.s32.b1.b1.s32.and.popc {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-                     : "+r"(acc[i][0]), "+r"(acc[i][1]), "+r"(acc[i][2]), "+r"(acc[i][3])
-                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-    }
-  }
-  int s = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) s += acc[i][0] + acc[i][1] + acc[i][2] + acc[i][3];
-  if (s == 0x7fffffff) sink[threadIdx.x] = s;   // keeps the loop alive
-}
-
 // Failure-detection self-test: one thread waits, with the library's bounded wait, on an
 // mbarrier that nothing ever arrives on. The wait must give up after kWaitTimeoutNs and
 // the kernel must return normally, leaving the context usable; it records the outcome
@@ -126,18 +98,6 @@ extern "C" int blprobe_wait_timeout(unsigned int* out_host, void* stream) {
   wait_timeout_kernel<<<1, 32, 0, st>>>(out);
   if (cudaGetLastError() != cudaSuccess) return -1;
   if (cudaMemcpyAsync(out_host, out, 2 * sizeof(unsigned int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return -1;
-  return cudaStreamSynchronize(st) == cudaSuccess ? 0 : -1;
-}
-
-// Warp-MMA probe: `kind` 2 (s8 m16n8k32) or 3 (b1 m16n8k256); `blocks` x 256 threads,
-// `iters` x 8 MMAs per warp. The caller times it. Returns 0 or -1.
-extern "C" int blprobe_warp_mma(int kind, int blocks, int iters, void* stream) {
-  static int* sink = nullptr;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (!sink && cudaMalloc(&sink, 1024 * sizeof(int)) != cudaSuccess) return -1;
-  if (kind == 2) warp_mma_kernel<2><<<blocks, 256, 0, st>>>(iters, sink);
-  else warp_mma_kernel<3><<<blocks, 256, 0, st>>>(iters, sink);
-  if (cudaGetLastError() != cudaSuccess) return -1;
   return cudaStreamSynchronize(st) == cudaSuccess ? 0 : -1;
 }
 

@@ -27,7 +27,7 @@ def test_exports_every_header_function(L):
 
 
 def test_abi_version(L):
-    assert L.bitlinear_abi_version() == 1
+    assert L.bitlinear_abi_version() == 2
 
 
 def _err(L):
@@ -105,18 +105,33 @@ def test_fwd_grouped_validation(L):
 
 
 def test_bwd_validation(L):
-    need = L.bitlinear_bwd_workspace_size(16, 896, 896, 1)
+    need = L.bitlinear_bwd_workspace_size(16, 896, 896, 1, 0)
     assert need == 896 * 896 * 2
-    assert L.bitlinear_bwd_workspace_size(16, 896, 896, 0) == 0
+    assert L.bitlinear_bwd_workspace_size(16, 896, 896, 0, 0) == 0
+    # the dequantised-X option adds a bf16 [t, k_in] buffer after the ternary matrix
+    assert L.bitlinear_bwd_workspace_size(16, 896, 896, 1, 1) == 896 * 896 * 2 + 16 * 896 * 2
+    assert L.bitlinear_bwd_workspace_size(16, 896, 896, 0, 1) == 16 * 896 * 2
+    #        dy    x     xq    absmax codes w_scale t  k_in n_out gx gw dtype flags ws  bytes stream
     # nothing requested
-    assert L.bitlinear_bwd(GOOD, GOOD, GOOD, GOOD, 16, 896, 896, None, None, 0, GOOD, need, None) == -1
+    assert L.bitlinear_bwd(GOOD, GOOD, None, None, GOOD, GOOD, 16, 896, 896, None, None, 0, 0, GOOD, need, None) == -1
     # grad_x without codes
-    assert L.bitlinear_bwd(GOOD, GOOD, None, GOOD, 16, 896, 896, GOOD, None, 0, GOOD, need, None) == -1
+    assert L.bitlinear_bwd(GOOD, GOOD, None, None, None, GOOD, 16, 896, 896, GOOD, None, 0, 0, GOOD, need, None) == -1
     # workspace too small for grad_x
-    assert L.bitlinear_bwd(GOOD, GOOD, GOOD, GOOD, 16, 896, 896, GOOD, None, 0, GOOD, need - 16, None) == -7
+    assert L.bitlinear_bwd(GOOD, GOOD, None, None, GOOD, GOOD, 16, 896, 896, GOOD, None, 0, 0, GOOD, need - 16,
+                           None) == -7
     # grad_w only needs no workspace; bad dtype is rejected
-    assert L.bitlinear_bwd(GOOD, GOOD, None, None, 16, 896, 896, None, GOOD, 3, None, 0, None) == -1
-    assert L.bitlinear_bwd(GOOD, BAD, None, None, 16, 896, 896, None, GOOD, 0, None, 0, None) == -3
+    assert L.bitlinear_bwd(GOOD, GOOD, None, None, None, None, 16, 896, 896, None, GOOD, 3, 0, None, 0, None) == -1
+    assert L.bitlinear_bwd(GOOD, BAD, None, None, None, None, 16, 896, 896, None, GOOD, 0, 0, None, 0, None) == -3
+    # unknown flag bits
+    assert L.bitlinear_bwd(GOOD, GOOD, None, None, None, None, 16, 896, 896, None, GOOD, 0, 2, None, 0, None) == -1
+    assert "flags" in _err(L)
+    # the dequantised-X option needs xq and absmax (x is not needed) and its workspace
+    deq = L.bitlinear_bwd_workspace_size(16, 896, 896, 0, 1)
+    assert L.bitlinear_bwd(GOOD, None, None, GOOD, None, None, 16, 896, 896, None, GOOD, 0, 1, GOOD, deq, None) == -1
+    assert L.bitlinear_bwd(GOOD, None, GOOD, None, None, None, 16, 896, 896, None, GOOD, 0, 1, GOOD, deq, None) == -1
+    assert L.bitlinear_bwd(GOOD, None, GOOD, GOOD, None, None, 16, 896, 896, None, GOOD, 0, 1, GOOD, deq - 16,
+                           None) == -7
+    assert L.bitlinear_bwd(GOOD, None, BAD, GOOD, None, None, 16, 896, 896, None, GOOD, 0, 1, GOOD, deq, None) == -3
 
 
 def test_grad_x_i8_validation(L):

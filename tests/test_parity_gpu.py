@@ -272,6 +272,43 @@ def test_grad_w_f32_and_masked_positions():
     assert torch.equal(g2, g8)
 
 
+@pytest.mark.parametrize("t,k_in,n_out,with_grad_x", [(200, 896, 256, False), (1000, 2048, 1024, True)])
+def test_grad_w_dequantised_x(t, k_in, n_out, with_grad_x):
+    """BL_GRADW_DEQUANT_X: grad_W against q * a / 127 (what the forward consumed),
+    alone and together with grad_X in one call (both buffers in one workspace)."""
+    w, x, dy = layer_inputs(1, 41, t, k_in, n_out)
+    ref_q, ref_a = O.act_quant(x)
+    xq, a = gpu_act_quant(x)
+    check_act_quant(xq, a, ref_q, ref_a, "dequant-x")
+    ref_qm = O.quant_mask(w, 6, 8)
+    qm = gpu_quant_mask(w, 6, 8)
+    gx, gw = B.bitlinear_bwd(bits_to_dev_bf16(dy), None, qm["codes"] if with_grad_x else None,
+                             qm["w_scale"] if with_grad_x else None, want_grad_x=with_grad_x, xq=xq, absmax=a,
+                             flags=B.BL_GRADW_DEQUANT_X)
+    torch.cuda.synchronize()
+    ref = O.grad_w(dy, x, x_deq=O.dequant_x(ref_q, ref_a))
+    assert_grad_close(bf16_dev_to_bits(gw), ref, "grad_w (dequantised x)")
+    # the two readings of X really differ here (1% x20 outliers): the option is not a no-op
+    raw = O.grad_w(dy, x)
+    assert np.max(np.abs(ref - raw)) / np.max(np.abs(raw)) > 2e-2
+    if with_grad_x:
+        assert_grad_close(bf16_dev_to_bits(gx), O.grad_x(dy, ref_qm["mcode"], ref_qm["gamma"]), "grad_x (same call)")
+
+
+def test_grad_w_dequantised_x_training_shape():
+    """Qwen2.5-3B gate shape, 16384 tokens, sampled output rows."""
+    t, k_in, n_out = 16384, 2048, 11008
+    _, x, dy = layer_inputs(4, 0, t, k_in, n_out)
+    ref_q, ref_a = O.act_quant(x)
+    xq, a = gpu_act_quant(x)
+    _, gw = B.bitlinear_bwd(bits_to_dev_bf16(dy), None, None, None, want_grad_x=False, xq=xq, absmax=a,
+                            flags=B.BL_GRADW_DEQUANT_X)
+    torch.cuda.synchronize()
+    rows = sample_rows(n_out, 5)
+    ref = O.grad_w(dy, x, rows=rows, x_deq=O.dequant_x(ref_q, ref_a))
+    assert_grad_close(bf16_dev_to_bits(gw)[rows], ref, "grad_w (dequantised x) training shape")
+
+
 def test_range_error_reported():
     w = synth.latent_weight(90, 64, 128)
     w[3, 5] = np.nan

@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import sparsity_step_b200 as B
+from oracle import bitlinear_oracle as O
 from sparsity_step_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -37,6 +38,34 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
         for key in ("codes", "mask", "w_i8"):
             assert torch.equal(got[key], ref[key]), key
         assert np.array_equal(got["w_scale"].cpu().numpy().view(np.uint32), ref["w_scale"].cpu().numpy().view(np.uint32))
+        # and directly against the oracle
+        want = O.quant_mask(w.cpu().numpy(), n, m)
+        assert np.array_equal(got["codes"].cpu().numpy(), want["codes_packed"])
+        assert np.array_equal(got["mask"].cpu().numpy(), want["mask"])
+        assert got["w_scale"].cpu().numpy()[0] == want["gamma"]
+
+
+def test_noalloc_range_error_then_clean_call():
+    """A non-finite weight gives gamma = NaN and all-zero codes; the next call on clean
+    weights is bit-exact again (the last block of each call resets the shared flag and
+    ticket in the built-in scratch)."""
+    dev = torch.device("cuda", 0)
+    n_out, k_in = 256, 896
+    w_np = synth.latent_weight(403, n_out, k_in)
+    bad = w_np.copy()
+    bad[7, 100] = np.inf
+    out = _outputs(n_out, k_in, 8, dev)
+    B.bitlinear_quant_mask_noalloc(torch.from_numpy(bad).to(dev), 6, 8, out=out)
+    torch.cuda.synchronize()
+    assert np.isnan(out["w_scale"].cpu().numpy()[0])
+    assert int(out["codes"].count_nonzero().item()) == 0
+    w = torch.from_numpy(w_np).to(dev)
+    got = B.bitlinear_quant_mask_noalloc(w, 6, 8, out=_outputs(n_out, k_in, 8, dev))
+    ref = B.bitlinear_quant_mask(w, 6, 8)
+    torch.cuda.synchronize()
+    for key in ("codes", "mask", "w_i8"):
+        assert torch.equal(got[key], ref[key]), key
+    assert got["w_scale"].cpu().numpy()[0] == O.quant_mask(w_np, 6, 8)["gamma"]
 
 
 def test_noalloc_rejects_oversize_tensor():
