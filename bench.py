@@ -430,7 +430,8 @@ def run_ours(args) -> None:
 
     # ---------------- raw tensor-pipe rates of this GPU (probe: MMAs from shared memory only)
     try:
-        probe = {"int8_tops": round(mma_peak("i8"), 1), "bf16_tflops": round(mma_peak("bf16"), 1)}
+        probe = {"int8_tops": round(mma_peak("i8"), 1), "bf16_tflops": round(mma_peak("bf16"), 1),
+                 "sparse_int8_tops_dense_equiv": round(mma_peak("sp_i8"), 1)}
     except (OSError, RuntimeError) as exc:
         probe = {"error": str(exc)}
 
@@ -620,8 +621,9 @@ def run_reference(args) -> None:
 
 
 def mma_peak(kind: str, iters: int = 4000, reps: int = 3) -> float:
-    """Dense tcgen05 MMA rate (TOP/s or TFLOP/s) of this GPU from the probe library:
-    148 CTAs issuing back-to-back 128x256 MMAs from shared memory (no memory traffic)."""
+    """tcgen05 MMA rate (TOP/s or TFLOP/s; dense-equivalent for the 2:4-sparse kind) of
+    this GPU from the probe library: 148 CTAs issuing back-to-back 128x256 MMAs from
+    shared memory (no memory traffic)."""
     import ctypes
 
     import torch
@@ -629,7 +631,7 @@ def mma_peak(kind: str, iters: int = 4000, reps: int = 3) -> float:
     lib = ctypes.CDLL(os.path.join(ROOT, "sparsity_step_b200", "libblprobe.so"))
     lib.blprobe_mma_peak.restype = ctypes.c_int
     lib.blprobe_mma_peak.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
-    k = 1 if kind == "i8" else 0
+    k = {"bf16": 0, "i8": 1, "sp_i8": 2}[kind]
     ctas = torch.cuda.get_device_properties(0).multi_processor_count
     st = torch.cuda.current_stream()
     if lib.blprobe_mma_peak(k, ctas, 100, st.cuda_stream) != 0:
@@ -643,7 +645,7 @@ def mma_peak(kind: str, iters: int = 4000, reps: int = 3) -> float:
         torch.cuda.synchronize()
         if rc != 0:
             raise RuntimeError(f"mma probe failed ({rc})")
-        kdim = 32 if kind == "i8" else 16
+        kdim = {"bf16": 16, "i8": 32, "sp_i8": 64}[kind]   # logical K per MMA
         ops = 2.0 * 128 * 256 * kdim * 4 * iters * ctas
         best = max(best, ops / (s.elapsed_time(e) * 1e-3) / 1e12)
     return best
@@ -659,7 +661,7 @@ def run_case(args) -> None:
     from sparsity_step_b200 import synth
 
     if args.case.startswith("mma_peak"):
-        kind = args.case.split("_")[-1]
+        kind = args.case[len("mma_peak_"):]
         print(json.dumps({"case": args.case, "rate": round(mma_peak(kind), 1),
                           "unit": "TOP/s" if kind == "i8" else "TFLOP/s"}), flush=True)
         return
@@ -673,6 +675,7 @@ def run_case(args) -> None:
     x = bf(synth.activation_bf16(12, t, k_in))
     dy = bf(synth.activation_bf16(13, t, n_out, std=1e-2, outliers=False))
     qm = B.bitlinear_quant_mask(w, N_KEEP, M_GROUP)
+    qm24 = B.bitlinear_quant_mask(w, 2, 4, want_sp=True) if args.case == "fwd_sp" else None
     xq, a = B.bitlinear_act_quant(x)
     y = torch.empty((t, n_out), dtype=torch.bfloat16, device=dev)
     gx = torch.empty((t, k_in), dtype=torch.bfloat16, device=dev)
@@ -687,6 +690,9 @@ def run_case(args) -> None:
                        "GB/s", n_out * k_in * (4 + 4 + 1 + 0.25 + 0.125)),
         "act_quant": (lambda: B.bitlinear_act_quant(x, xq=xq, absmax=a), "GB/s", t * k_in * 3 + 4 * t),
         "fwd": (lambda: B.bitlinear_fwd(xq, a, qm["w_scale"], w_i8=qm["w_i8"], y=y), "TOP/s", flops),
+        # 2:4 mask on the sparse tensor cores: dense-equivalent ops
+        "fwd_sp": (lambda: B.bitlinear_fwd(xq, a, qm24["w_scale"], sp_values=qm24["sp_values"], sp_meta=qm24["sp_meta"],
+                                           y=y), "TOP/s", flops),
         "fwd_codes": (lambda: B.bitlinear_fwd(xq, a, qm["w_scale"], codes=qm["codes"], y=y), "GB/s",
                       n_out * k_in / 4 + t * k_in + 2 * t * n_out),
         "grad_x": (lambda: B.bitlinear_bwd(dy, None, qm["codes"], qm["w_scale"], want_grad_w=False, grad_x=gx,
@@ -825,7 +831,8 @@ def run_decode(args) -> None:
     dev = torch.device("cuda", 0)
     peaks = load_peaks()
     n_keep, m_group = (8, 8) if args.dense else (N_KEEP, M_GROUP)
-    layers, code_bytes = build_decode_stack(dev, n_keep, m_group, distinct=True, want_w_i8=args.prefill > 0)
+    layers, code_bytes = build_decode_stack(dev, n_keep, m_group, distinct=not args.clone_layers,
+                                            want_w_i8=args.prefill > 0)
     res = {"workload": "Qwen2.5-3B-shaped 36-layer BitLinear stack, forward",
            "nm": f"{n_keep}:{m_group}", "code_bytes_per_step": code_bytes,
            "hbm_peak_gbs": peaks["hbm_gbs"],
@@ -894,20 +901,27 @@ def measure_sweep(steps: int, warmup: int, nms=None) -> dict:
             y = torch.empty((t, n_out), dtype=torch.bfloat16, device=dev)
             row = {}
             for n, m in (nms or SWEEP_NM):
-                qm = B.bitlinear_quant_mask(w, n, m)
-                for _ in range(warmup):
-                    B.bitlinear_fwd(xq, a, qm["w_scale"], w_i8=qm["w_i8"], y=y)
-                torch.cuda.synchronize()
-                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                s.record()
-                for _ in range(steps):
-                    B.bitlinear_fwd(xq, a, qm["w_scale"], w_i8=qm["w_i8"], y=y)
-                e.record()
-                torch.cuda.synchronize()
-                ms = s.elapsed_time(e) / steps
-                ops = 2.0 * t * k_in * n_out
-                row[f"{n}:{m}"] = {"us": round(ms * 1e3, 2), "tops_dense_equiv": round(ops / (ms * 1e-3) / 1e12, 1),
-                                   "tops_useful": round(ops * n / m / (ms * 1e-3) / 1e12, 1)}
+                # masks with at most two kept per aligned four also run on the sparse
+                # tensor cores ("n:m sparse"); every mask runs on the dense int8 path
+                sparse_ok = n <= 2 and k_in % 128 == 0
+                qm = B.bitlinear_quant_mask(w, n, m, want_sp=sparse_ok)
+                variants = [(f"{n}:{m}", {"w_i8": qm["w_i8"]})]
+                if sparse_ok:
+                    variants.append((f"{n}:{m} sparse", {"sp_values": qm["sp_values"], "sp_meta": qm["sp_meta"]}))
+                for key, kw in variants:
+                    for _ in range(warmup):
+                        B.bitlinear_fwd(xq, a, qm["w_scale"], y=y, **kw)
+                    torch.cuda.synchronize()
+                    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    s.record()
+                    for _ in range(steps):
+                        B.bitlinear_fwd(xq, a, qm["w_scale"], y=y, **kw)
+                    e.record()
+                    torch.cuda.synchronize()
+                    ms = s.elapsed_time(e) / steps
+                    ops = 2.0 * t * k_in * n_out
+                    row[key] = {"us": round(ms * 1e3, 2), "tops_dense_equiv": round(ops / (ms * 1e-3) / 1e12, 1),
+                                "tops_useful": round(ops * n / m / (ms * 1e-3) / 1e12, 1)}
             base = row["8:8"]["us"]
             for k in row:
                 row[k]["speedup_vs_8_8"] = round(base / row[k]["us"], 4)
@@ -929,9 +943,8 @@ def main(argv=None) -> None:
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the N:M sweep and decode sub-records")
-    ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_codes", "grad_x", "grad_w", "grad_x_i8",
-                                       "mask_hist", "mma_peak_i8",
-                                       "mma_peak_bf16"],
+    ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_sp", "fwd_codes", "grad_x", "grad_w",
+                                       "grad_x_i8", "mask_hist", "mma_peak_i8", "mma_peak_bf16", "mma_peak_sp_i8"],
                     help="time one kernel class alone on the --case-t/k/n shape")
     ap.add_argument("--case-t", type=int, default=TOKENS)
     ap.add_argument("--case-k", type=int, default=2048)
@@ -941,6 +954,8 @@ def main(argv=None) -> None:
     ap.add_argument("--batches", type=int, nargs="+", default=[1, 8, 32, 128])
     ap.add_argument("--prefill", type=int, default=8192, help="prefill tokens for --workload decode (0 = skip)")
     ap.add_argument("--dense", action="store_true", help="--workload decode with 8:8 (no mask)")
+    ap.add_argument("--clone-layers", action="store_true",
+                    help="--workload decode: generate layer 0 and copy its codes into the other 35 layers' buffers")
     args = ap.parse_args(argv)
     if args.workload == "decode":
         run_decode(args)

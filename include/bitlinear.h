@@ -80,6 +80,19 @@ size_t bitlinear_quant_mask_workspace_size(int64_t n_out, int64_t k_in);
  *                at bits 2*(k % 4) of byte k / 4; 00 = 0, 01 = +1, 11 = -1.
  *   w_i8_out     [n_out, k_in] int8, out, nullable. Masked codes as int8 (the
  *                operand of the tensor-core forward product).
+ *   sp_values_out [n_out, k_in / 2] int8, out, nullable, and
+ *   sp_meta_out  [n_sp, k_sp / 8] uint8, out, nullable, with n_sp = n_out and k_sp =
+ *                k_in each rounded up to a multiple of 256 (both or neither; only for
+ *                masks with at most two kept weights in every aligned group of four:
+ *                n_keep <= 2, else BL_ERR_INVALID_ARG). The 2:4 structured form of the
+ *                masked codes that sparse tensor cores take (Sparse-BitNet article,
+ *                section 七: NVIDIA's sparse tensor cores need the 2:4 pattern): per
+ *                aligned group of four, two stored values and their positions i0 < i1
+ *                (the kept positions, completed with the lowest unused ones, whose
+ *                value is 0). Values of group g at bytes 2g, 2g+1 of the row; metadata
+ *                nibble i0 | i1 << 2 of group g in bits 4*(g % 2) of byte g / 2 of the
+ *                row. The padding rows and columns of sp_meta hold 0x44 (positions 0
+ *                and 1), so that the sparse product reads whole tiles of valid metadata.
  *   w_scale_out  [1] fp32, out: gamma. NaN when the range check fails.
  *   workspace    bitlinear_quant_mask_workspace_size() bytes, scratch, in/out.
  *
@@ -88,8 +101,9 @@ size_t bitlinear_quant_mask_workspace_size(int64_t n_out, int64_t k_in);
  * Calls that share a workspace must not overlap on the GPU.
  */
 bl_status bitlinear_quant_mask(const float* w_latent, int64_t n_out, int64_t k_in, int n_keep, int m_group,
-                               uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out, float* w_scale_out,
-                               void* workspace, size_t workspace_bytes, void* stream);
+                               uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out, int8_t* sp_values_out,
+                               uint8_t* sp_meta_out, float* w_scale_out, void* workspace, size_t workspace_bytes,
+                               void* stream);
 
 /* Synchronises `stream`, then returns the range status (BL_OK or BL_ERR_RANGE) that
  * the last bitlinear_quant_mask using `workspace` recorded. */
@@ -103,7 +117,7 @@ bl_status bitlinear_quant_mask_status(const void* workspace, void* stream);
  * (which may synchronise the device) are not allowed.
  *
  * Same computation, arguments and outputs as bitlinear_quant_mask, minus the
- * workspace. Its scratch is a fixed array of 19200 bytes inside the library (every
+ * workspace and the 2:4 outputs. Its scratch is a fixed array of 19200 bytes inside the library (every
  * GPU that loads the library holds it until exit), which limits the tensor to
  * n_out * k_in <= 4966055936 weights; larger tensors get BL_ERR_UNSUPPORTED_SHAPE.
  * The first call on each device looks up that array's device address (with the
@@ -135,10 +149,17 @@ bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t
  *   y[t, n]   = acc * (absmax[t] / 127 * gamma)              (fp32, then bf16 or f32)
  *
  *   xq [t, k_in] int8, absmax [t] fp32 (from bitlinear_act_quant).
- *   codes [n_out, k_in / 4] (packed masked codes), w_i8 [n_out, k_in] int8 (masked
- *   codes): give at least one. With w_i8 the product runs on the tcgen05 int8 tensor
- *   cores (TMA-fed, for prefill and training shapes); with codes only it streams the
- *   2-bit codes and decodes them into register MMA fragments (for decode batches).
+ *   The masked weights, in one of three forms (give at least one; the first given
+ *   in this order is used):
+ *     sp_values [n_out, k_in / 2] int8 + sp_meta [n_sp, k_sp / 8] uint8 (padded, see
+ *       bitlinear_quant_mask): the 2:4 form from bitlinear_quant_mask (masks with at
+ *       most two kept per aligned four). Runs on the sparse tensor cores
+ *       (tcgen05.mma.sp kind::i8, CTA pairs): Sparse-BitNet article, section 七.
+ *     w_i8 [n_out, k_in] int8 masked codes: the dense tcgen05 int8 tensor cores
+ *       (TMA-fed, for prefill and training shapes).
+ *     codes [n_out, k_in / 4] packed masked codes: streams the 2-bit codes and
+ *       decodes them on chip (for decode batches): BitNet b1.58 2B4T article,
+ *       section 四.
  *   w_scale [1] fp32 gamma. acc_out [t, n_out] int32, out, nullable.
  *   y_out [t, n_out], out, bf16 (y_dtype = BL_OUT_BF16) or fp32 (BL_OUT_F32).
  * No bias term.
@@ -148,8 +169,8 @@ bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t
  * table does not fit, every such call returns BL_ERR_CUDA before enqueueing anything.
  */
 bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* codes, const int8_t* w_i8,
-                        const float* w_scale, int64_t t, int64_t k_in, int64_t n_out, int32_t* acc_out, void* y_out,
-                        int y_dtype, void* stream);
+                        const int8_t* sp_values, const uint8_t* sp_meta, const float* w_scale, int64_t t, int64_t k_in,
+                        int64_t n_out, int32_t* acc_out, void* y_out, int y_dtype, void* stream);
 
 /* One forward problem of bitlinear_fwd_grouped (same meaning as the arguments of
  * bitlinear_fwd, codes operand only). */

@@ -300,6 +300,20 @@ def dequant_x(q: np.ndarray, absmax: np.ndarray) -> np.ndarray:
     return q.astype(np.float64) * (absmax.astype(np.float64)[:, None] / 127.0)
 
 
+def dequant_x_bf16(q: np.ndarray, absmax: np.ndarray) -> np.ndarray:
+    """X_deq as a bf16 operand (fp64 values of the bf16 numbers): s_t = fp32(a_t / 127),
+    one fp32 multiply q * s_t, then round to the nearest bf16 (ties to even).
+
+    reading: the dequantised-activation option of grad_W feeds a bf16 product, so its
+    operand is X_deq rounded to bf16; ``dequant_x`` is the exact value it rounds.
+    """
+    s = (np.asarray(absmax, dtype=np.float32) / np.float32(127.0)).astype(np.float32)
+    p = (np.asarray(q, dtype=np.float32) * s[:, None]).astype(np.float32)
+    u = p.view(np.uint32).astype(np.uint64)
+    r = ((u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)).astype(np.uint32)
+    return (r << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
 def grad_x_int8_dy(dy_bits: np.ndarray, mcode: np.ndarray, gamma: np.float32,
                    rows: np.ndarray | None = None) -> tuple[np.ndarray, np.ndarray, np.ndarray, np.ndarray]:
     """grad_X with dY quantised per token to int8, as an exact integer product.

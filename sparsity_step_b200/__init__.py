@@ -4,6 +4,7 @@ The functions below are thin bindings of the C ABI in include/bitlinear.h; the
 library libbitlinear.so is loaded on first use and its absence is an error.
 """
 from .bitlinear import (  # noqa: F401
+    BL_GRADW_DEQUANT_X,
     BL_OUT_BF16,
     BL_OUT_F32,
     bitlinear_abi_version,
@@ -20,4 +21,5 @@ from .bitlinear import (  # noqa: F401
     bitlinear_quant_mask_noalloc,
     bitlinear_quant_mask_status,
     bitlinear_quant_mask_workspace_size,
+    sp_meta_shape,
 )

@@ -37,11 +37,11 @@ class BlFwdProblem(ctypes.Structure):
 # name -> (restype, argtypes), in the order of include/bitlinear.h
 SIGNATURES = {
     "bitlinear_quant_mask_workspace_size": (_SZ, [_I64, _I64]),
-    "bitlinear_quant_mask": (_INT, [_P, _I64, _I64, _INT, _INT, _P, _P, _P, _P, _P, _SZ, _P]),
+    "bitlinear_quant_mask": (_INT, [_P, _I64, _I64, _INT, _INT, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bitlinear_quant_mask_status": (_INT, [_P, _P]),
     "bitlinear_quant_mask_noalloc": (_INT, [_P, _I64, _I64, _INT, _INT, _P, _P, _P, _P, _P]),
     "bitlinear_act_quant": (_INT, [_P, _I64, _I64, _P, _P, _P]),
-    "bitlinear_fwd": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P]),
+    "bitlinear_fwd": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P]),
     "bitlinear_fwd_grouped": (_INT, [_c.POINTER(BlFwdProblem), _INT, _INT, _P]),
     "bitlinear_bwd_workspace_size": (_SZ, [_I64, _I64, _I64, _INT, _INT]),
     "bitlinear_bwd": (_INT, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _INT, _P, _SZ, _P]),

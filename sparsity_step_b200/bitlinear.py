@@ -55,6 +55,11 @@ def _need_bytes(t, nbytes, name, device=None):
     return _need_vec(t, torch.uint8, nbytes, name, device)
 
 
+def sp_meta_shape(n_out: int, k_in: int) -> tuple[int, int]:
+    """Shape of the padded 2:4 metadata: rows and logical K rounded up to 256."""
+    return (n_out + 255) // 256 * 256, (k_in + 255) // 256 * 256 // 8
+
+
 def _check_qm_outputs(o: dict, n_out: int, k_in: int, m_group: int, dev) -> None:
     _need(o["codes"], torch.uint8, (n_out, k_in // 4), "codes", dev)
     _need_vec(o["w_scale"], torch.float32, 1, "w_scale", dev)
@@ -62,6 +67,9 @@ def _check_qm_outputs(o: dict, n_out: int, k_in: int, m_group: int, dev) -> None
         _need(o["mask"], torch.uint8, (n_out, k_in // m_group), "mask", dev)
     if o.get("w_i8") is not None:
         _need(o["w_i8"], torch.int8, (n_out, k_in), "w_i8", dev)
+    if o.get("sp_values") is not None or o.get("sp_meta") is not None:
+        _need(o["sp_values"], torch.int8, (n_out, k_in // 2), "sp_values", dev)
+        _need(o["sp_meta"], torch.uint8, sp_meta_shape(n_out, k_in), "sp_meta", dev)
 
 
 def bitlinear_quant_mask_workspace_size(n_out: int, k_in: int) -> int:
@@ -69,12 +77,14 @@ def bitlinear_quant_mask_workspace_size(n_out: int, k_in: int) -> int:
 
 
 def bitlinear_quant_mask(w: torch.Tensor, n_keep: int, m_group: int, *, want_mask: bool = True,
-                         want_w_i8: bool = True, out: dict | None = None, workspace: torch.Tensor | None = None,
-                         stream=None) -> dict:
+                         want_w_i8: bool = True, want_sp: bool = False, out: dict | None = None,
+                         workspace: torch.Tensor | None = None, stream=None) -> dict:
     """Mask, gamma and masked ternary codes of latent weights w [n_out, k_in] (fp32).
 
     Returns a dict with ``codes`` (uint8 [n_out, k_in/4]), ``w_scale`` (fp32 [1]),
-    and optionally ``mask`` (uint8 [n_out, k_in/m]) and ``w_i8`` (int8 [n_out, k_in]).
+    and optionally ``mask`` (uint8 [n_out, k_in/m]), ``w_i8`` (int8 [n_out, k_in]) and,
+    for masks with at most two kept per aligned four (``want_sp``), the 2:4 form
+    ``sp_values`` (int8 [n_out, k_in/2]) and ``sp_meta`` (uint8, padded: ``sp_meta_shape``).
     """
     n_out, k_in = w.shape
     _need(w, torch.float32, None, "w")
@@ -88,6 +98,9 @@ def bitlinear_quant_mask(w: torch.Tensor, n_keep: int, m_group: int, *, want_mas
         o["mask"] = torch.empty((n_out, k_in // m_group), dtype=torch.uint8, device=dev)
     if want_w_i8 and "w_i8" not in o:
         o["w_i8"] = torch.empty((n_out, k_in), dtype=torch.int8, device=dev)
+    if want_sp and "sp_values" not in o:
+        o["sp_values"] = torch.empty((n_out, k_in // 2), dtype=torch.int8, device=dev)
+        o["sp_meta"] = torch.empty(sp_meta_shape(n_out, k_in), dtype=torch.uint8, device=dev)
     if m_group not in (4, 8) or k_in % m_group:
         raise ValueError(f"m_group must be 4 or 8 and divide k_in (got {m_group})")
     _check_qm_outputs(o, n_out, k_in, m_group, dev)
@@ -96,8 +109,8 @@ def bitlinear_quant_mask(w: torch.Tensor, n_keep: int, m_group: int, *, want_mas
         workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
     _need_bytes(workspace, ws_bytes, "workspace", dev)
     st = lib().bitlinear_quant_mask(_ptr(w), n_out, k_in, n_keep, m_group, _ptr(o.get("mask")), _ptr(o["codes"]),
-                                    _ptr(o.get("w_i8")), _ptr(o["w_scale"]), _ptr(workspace), workspace.numel(),
-                                    _stream(stream))
+                                    _ptr(o.get("w_i8")), _ptr(o.get("sp_values")), _ptr(o.get("sp_meta")),
+                                    _ptr(o["w_scale"]), _ptr(workspace), workspace.numel(), _stream(stream))
     check(st, "bitlinear_quant_mask")
     o["workspace"] = workspace
     return o
@@ -145,17 +158,26 @@ def bitlinear_act_quant(x: torch.Tensor, *, xq: torch.Tensor | None = None, absm
 
 
 def bitlinear_fwd(xq: torch.Tensor, absmax: torch.Tensor, w_scale: torch.Tensor, *, codes: torch.Tensor | None = None,
-                  w_i8: torch.Tensor | None = None, n_out: int | None = None, y_dtype=torch.bfloat16,
+                  w_i8: torch.Tensor | None = None, sp_values: torch.Tensor | None = None,
+                  sp_meta: torch.Tensor | None = None, n_out: int | None = None, y_dtype=torch.bfloat16,
                   want_acc: bool = False, y: torch.Tensor | None = None, acc: torch.Tensor | None = None,
                   stream=None) -> tuple[torch.Tensor, torch.Tensor | None]:
-    """y = (xq . masked_codes^T) * absmax/127 * gamma; returns (y, acc or None)."""
+    """y = (xq . masked_codes^T) * absmax/127 * gamma; returns (y, acc or None).
+
+    Weight operand: the 2:4 form (``sp_values`` + ``sp_meta``, sparse tensor cores),
+    else ``w_i8`` (dense tensor cores), else ``codes`` (2-bit codes decoded on chip)."""
     t, k_in = xq.shape
     dev = xq.device
     _need(xq, torch.int8, None, "xq")
-    if w_i8 is None and codes is None:
-        raise ValueError("give codes or w_i8")
+    if w_i8 is None and codes is None and sp_values is None:
+        raise ValueError("give codes, w_i8 or sp_values + sp_meta")
+    if (sp_values is None) != (sp_meta is None):
+        raise ValueError("give both sp_values and sp_meta, or neither")
     if n_out is None:
-        n_out = (w_i8 if w_i8 is not None else codes).shape[0]
+        n_out = (sp_values if sp_values is not None else w_i8 if w_i8 is not None else codes).shape[0]
+    if sp_values is not None:
+        _need(sp_values, torch.int8, (n_out, k_in // 2), "sp_values", dev)
+        _need(sp_meta, torch.uint8, sp_meta_shape(n_out, k_in), "sp_meta", dev)
     if codes is not None:
         _need(codes, torch.uint8, (n_out, k_in // 4), "codes", dev)
     if w_i8 is not None:
@@ -172,8 +194,8 @@ def bitlinear_fwd(xq: torch.Tensor, absmax: torch.Tensor, w_scale: torch.Tensor,
     if acc is not None:
         _need(acc, torch.int32, (t, n_out), "acc", dev)
     ydt = BL_OUT_F32 if y.dtype == torch.float32 else BL_OUT_BF16
-    st = lib().bitlinear_fwd(_ptr(xq), _ptr(absmax), _ptr(codes), _ptr(w_i8), _ptr(w_scale), t, k_in, n_out,
-                             _ptr(acc), _ptr(y), ydt, _stream(stream))
+    st = lib().bitlinear_fwd(_ptr(xq), _ptr(absmax), _ptr(codes), _ptr(w_i8), _ptr(sp_values), _ptr(sp_meta),
+                             _ptr(w_scale), t, k_in, n_out, _ptr(acc), _ptr(y), ydt, _stream(stream))
     check(st, "bitlinear_fwd")
     return y, acc
 
@@ -340,6 +362,6 @@ __all__ = [
     "bitlinear_quant_mask_workspace_size", "bitlinear_quant_mask", "bitlinear_quant_mask_status",
     "bitlinear_quant_mask_noalloc",
     "bitlinear_act_quant", "bitlinear_fwd", "bitlinear_fwd_grouped", "bitlinear_bwd_workspace_size", "bitlinear_bwd",
-    "bitlinear_grad_x_i8_workspace_size", "bitlinear_grad_x_i8", "bitlinear_mask_threshold_hist",
+    "bitlinear_grad_x_i8_workspace_size", "bitlinear_grad_x_i8", "bitlinear_mask_threshold_hist", "sp_meta_shape",
     "bitlinear_device_status", "bitlinear_abi_version", "BL_OUT_BF16", "BL_OUT_F32", "BL_GRADW_DEQUANT_X", "_lib",
 ]

@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "diag_kernels.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_sp2.cuh"
 #include "gemm_tc2.cuh"
 #include "quant_mask.cuh"
 
@@ -70,9 +71,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D row-major tensor [outer, inner], 128-byte swizzled boxes of [box_outer, box_inner].
+// 2-D row-major tensor [outer, inner], boxes of [box_outer, box_inner], 128-byte
+// swizzled unless `swizzle` is false.
 bl_status make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* base, uint64_t inner, uint64_t outer,
-                   uint32_t box_inner, uint32_t box_outer) {
+                   uint32_t box_inner, uint32_t box_outer, bool swizzle = true) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(BL_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {inner, outer};
@@ -80,7 +82,8 @@ bl_status make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const vo
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(BL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return BL_OK;
 }
@@ -154,6 +157,20 @@ bl_status launch_gemm2(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
 // Pairs pay off once the output has at least two 128-row blocks; a single block would
 // leave half of each pair's tensor work on rows outside the output.
 inline bool use_cta_pair(int64_t m) { return m > bl::kBM; }
+
+// Raster order of one product. By default tiles walk n blocks fastest (every wave
+// re-reads all of B). When B is larger than L2 and A is small enough to stay there, m
+// blocks go fastest instead, so that A is re-read from L2 and B streams once (grad_W of
+// the down projection: X [16384 x 11008] bf16 is 360 MB; measured 1.91 -> 0.72 GB of
+// DRAM reads per launch). No eviction hints: marking the streamed operand evict-first
+// doubled the DRAM reads (its lines left L2 before the other tiles of the same wave
+// read them).
+void set_raster(bl::GemmArgs& g, double a_bytes, double b_bytes) {
+  constexpr double kL2Bytes = 96e6;   // usable share of the 126 MB L2
+  g.m_fastest = (b_bytes > kL2Bytes && a_bytes < b_bytes && a_bytes <= 0.7 * kL2Bytes) ? 1 : 0;
+  g.a_l2 = bl::L2_NORMAL;
+  g.b_l2 = bl::L2_NORMAL;
+}
 
 // ------------------------------------------------------------------ grouped codes product
 
@@ -306,65 +323,125 @@ bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32
 
 // ------------------------------------------------------------------ quant_mask launches
 
+struct QmOutputs {
+  uint8_t* mask;
+  uint8_t* codes;
+  int8_t* w_i8;
+  int8_t* sp_values;
+  uint8_t* sp_meta;
+  int64_t k8, meta_pitch;   // metadata bytes per row and its padded row pitch
+};
+
+// Padded extents of the 2:4 metadata: rows and logical K rounded up to 256, so that the
+// sparse product's metadata loads never leave the tensor.
+inline int64_t sp_rows(int64_t n_out) { return (n_out + bl::kSpPad - 1) / bl::kSpPad * bl::kSpPad; }
+inline int64_t sp_meta_pitch(int64_t k_in) { return (k_in + bl::kSpPad - 1) / bl::kSpPad * bl::kSpPad / 8; }
+
 template <int M, int NK>
-void launch_mask_codes(const float* w, int64_t n8, int n_keep, const float* gamma, uint8_t* mask, uint8_t* codes,
-                       int8_t* w_i8, int grid, cudaStream_t st) {
-  bl::qm_mask_codes_kernel<M, NK><<<grid, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w), n8, n_keep, gamma,
-                                                                     mask, reinterpret_cast<uint16_t*>(codes),
-                                                                     reinterpret_cast<uint2*>(w_i8));
+void launch_mask_codes(const float* w, int64_t n8, int n_keep, const float* gamma, const QmOutputs& o, int grid,
+                       cudaStream_t st) {
+  bl::qm_mask_codes_kernel<M, NK><<<grid, bl::kQmThreads, 0, st>>>(
+      reinterpret_cast<const float4*>(w), n8, n_keep, gamma, o.mask, reinterpret_cast<uint16_t*>(o.codes),
+      reinterpret_cast<uint2*>(o.w_i8), reinterpret_cast<uint32_t*>(o.sp_values), o.sp_meta, o.k8, o.meta_pitch);
 }
 
 int qm_blocks(int64_t numel);
+int qm_blocks_launch(int64_t numel, int resident);
 
-// Both passes of steps a1 + a2 on `scratch` (its first 16 bytes are cleared here).
-bl_status enqueue_quant_mask(const float* w, int64_t n_out, int64_t k_in, int n_keep, int m_group, uint8_t* mask,
-                             uint8_t* codes, int8_t* w_i8, float* gamma, void* scratch, cudaStream_t st) {
+// Resident 256-thread blocks per SM of a kernel (registers decide it here), looked up
+// once per kernel; 1 if the query fails.
+template <typename K>
+int resident_blocks(K kern, int* cache) {
+  if (*cache <= 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, bl::kQmThreads, 0) != cudaSuccess || n <= 0) n = 1;
+    *cache = n;
+  }
+  return *cache;
+}
+
+// Both passes of steps a1 + a2 on `scratch` (its first 16 bytes are cleared here). Both
+// grids are one wave of resident blocks (grid-stride loops): a partial second wave
+// would leave most SMs idle at the end of each pass.
+bl_status enqueue_quant_mask(const float* w, int64_t n_out, int64_t k_in, int n_keep, int m_group, const QmOutputs& o,
+                             float* gamma, void* scratch, cudaStream_t st) {
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   cudaError_t e = cudaMemsetAsync(ws, 0, 16, st);   // range flag, status, blocks-done ticket
   if (e != cudaSuccess) return cuda_fail(e, "scratch reset");
   const int64_t numel = n_out * k_in;
-  const int blocks = qm_blocks(numel);
+  static int occ_sum = 0;
+  const int blocks = qm_blocks_launch(numel, device_sm_count() * resident_blocks(bl::qm_abs_sum_kernel, &occ_sum));
   bl::QmScratch q{reinterpret_cast<unsigned int*>(ws), reinterpret_cast<int*>(ws + 4),
                   reinterpret_cast<unsigned int*>(ws + 8), reinterpret_cast<unsigned long long*>(ws + bl::kQmWsHeader)};
   bl::qm_abs_sum_kernel<<<blocks, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w), numel / 4, numel, q, gamma);
   const int64_t n8 = numel / 8;
   int64_t g2 = (n8 + bl::kQmThreads - 1) / bl::kQmThreads;
-  const int64_t cap = int64_t(device_sm_count()) * 16;
+  static int occ_mask = 0;   // the same for every instantiation in practice (38-40 registers)
+  const int64_t cap = int64_t(device_sm_count()) * resident_blocks(bl::qm_mask_codes_kernel<8, 6>, &occ_mask);
   if (g2 > cap) g2 = cap;
   const int grid = static_cast<int>(g2);
   if (m_group == 8) {
     switch (n_keep) {
-      case 8: launch_mask_codes<8, 8>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
-      case 6: launch_mask_codes<8, 6>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
-      case 4: launch_mask_codes<8, 4>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
-      case 2: launch_mask_codes<8, 2>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
-      default: launch_mask_codes<8, 0>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+      case 8: launch_mask_codes<8, 8>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 7: launch_mask_codes<8, 7>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 6: launch_mask_codes<8, 6>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 5: launch_mask_codes<8, 5>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 4: launch_mask_codes<8, 4>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 3: launch_mask_codes<8, 3>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 2: launch_mask_codes<8, 2>(w, n8, n_keep, gamma, o, grid, st); break;
+      default: launch_mask_codes<8, 1>(w, n8, n_keep, gamma, o, grid, st); break;
     }
   } else {
     switch (n_keep) {
-      case 4: launch_mask_codes<4, 4>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
-      case 2: launch_mask_codes<4, 2>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
-      default: launch_mask_codes<4, 0>(w, n8, n_keep, gamma, mask, codes, w_i8, grid, st); break;
+      case 4: launch_mask_codes<4, 4>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 3: launch_mask_codes<4, 3>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 2: launch_mask_codes<4, 2>(w, n8, n_keep, gamma, o, grid, st); break;
+      default: launch_mask_codes<4, 1>(w, n8, n_keep, gamma, o, grid, st); break;
     }
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quant_mask launch");
+  if (o.sp_meta != nullptr) {   // padding: the valid pattern 0x4 in every group (positions 0, 1)
+    if (o.meta_pitch > o.k8) {
+      e = cudaMemset2DAsync(o.sp_meta + o.k8, static_cast<size_t>(o.meta_pitch), 0x44,
+                            static_cast<size_t>(o.meta_pitch - o.k8), static_cast<size_t>(n_out), st);
+      if (e != cudaSuccess) return cuda_fail(e, "metadata column padding");
+    }
+    const int64_t pad_rows = sp_rows(n_out) - n_out;
+    if (pad_rows > 0) {
+      e = cudaMemsetAsync(o.sp_meta + n_out * o.meta_pitch, 0x44, static_cast<size_t>(pad_rows * o.meta_pitch), st);
+      if (e != cudaSuccess) return cuda_fail(e, "metadata row padding");
+    }
+  }
   return BL_OK;
 }
 
 // ------------------------------------------------------------------ quant_mask sizing
 
+// Upper bound on the blocks of the sum pass (sizes the workspace: one 16-byte partial per
+// block): enough to fill 148 SMs with 8 blocks each, and enough that no thread sums more
+// than kQmMaxElemsPerThread weights.
 constexpr int kQmTargetBlocks = 148 * 8;
 
-int qm_blocks(int64_t numel) {
+int qm_blocks_bounded(int64_t numel, int64_t target) {
   const int64_t n4 = numel / 4;
   int64_t need = (numel + (int64_t(bl::kQmThreads) * bl::kQmMaxElemsPerThread) - 1) /
                  (int64_t(bl::kQmThreads) * bl::kQmMaxElemsPerThread);   // bounds elements per thread
   int64_t fill = (n4 + bl::kQmThreads - 1) / bl::kQmThreads;
-  if (fill > kQmTargetBlocks) fill = kQmTargetBlocks;
+  if (fill > target) fill = target;
   int64_t b = need > fill ? need : fill;
   if (b < 1) b = 1;
   return static_cast<int>(b);
+}
+
+int qm_blocks(int64_t numel) { return qm_blocks_bounded(numel, kQmTargetBlocks); }
+
+// Blocks actually launched: one wave of `resident` blocks (never more than the
+// workspace bound).
+int qm_blocks_launch(int64_t numel, int resident) {
+  const int b = qm_blocks_bounded(numel, resident < kQmTargetBlocks ? resident : kQmTargetBlocks);
+  const int bound = qm_blocks(numel);
+  return b < bound ? b : bound;
 }
 
 // Launch of the act_quant kernels (arguments already checked).
@@ -414,6 +491,7 @@ bl_status enqueue_fwd_i8(const int8_t* xq, const float* absmax, const int8_t* w_
   g.acc_out = acc_out;
   g.row_absmax = absmax;
   g.w_scale = w_scale;
+  set_raster(g, double(t) * double(k_in), double(n_out) * double(k_in));
   if (acc_out) {   // int32 accumulators requested: per-row direct stores of y and acc
     return launch_gemm<true, false, false, bl::EPI_FWD, false>(ta, tb, ta, g, st);
   }
@@ -429,6 +507,70 @@ bl_status enqueue_fwd_i8(const int8_t* xq, const float* absmax, const int8_t* w_
     if (launched) return BL_OK;
   }
   return launch_gemm<true, false, false, bl::EPI_FWD, true>(ta, tb, to, g, st);
+}
+
+// The 2:4 sparse product on CTA pairs (weights on M, tokens on N; arguments checked,
+// k_in % 128 == 0).
+bl_status enqueue_fwd_sp(const int8_t* xq, const float* absmax, const int8_t* sp_values, const uint8_t* sp_meta,
+                         const float* w_scale, int64_t t, int64_t k_in, int64_t n_out, int32_t* acc_out, void* y_out,
+                         bool y_f32, cudaStream_t st) {
+  CUtensorMap ta, tb, te;
+  if (bl_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sp_values, k_in / 2, n_out, 128, 128)) return s;
+  if (bl_status s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, k_in, t, 128, bl::kSpTokHalf)) return s;
+  if (bl_status s = make_map(&te, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sp_meta, sp_meta_pitch(k_in), sp_rows(n_out), 16,
+                             128, false))
+    return s;
+  CUtensorMap ty;
+  const bool tma_store = acc_out == nullptr;
+  if (tma_store) {
+    if (bl_status s = make_map(&ty, y_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                               y_f32 ? 4 : 2, y_out, n_out, t, 32, 16, false))
+      return s;
+  } else {
+    ty = te;   // unused
+  }
+  bl::SpGemmArgs g{};
+  g.tma_store = tma_store ? 1 : 0;
+  g.T = static_cast<int>(t);
+  g.n_out = static_cast<int>(n_out);
+  g.k_in = static_cast<int>(k_in);
+  g.num_k_blocks = static_cast<int>((k_in + bl::kSpKStep - 1) / bl::kSpKStep);
+  g.num_row_blocks = static_cast<int>((n_out + bl::kSpRowsPair - 1) / bl::kSpRowsPair);
+  g.num_tok_blocks = static_cast<int>((t + bl::kSpTok - 1) / bl::kSpTok);
+  g.y = y_out;
+  g.y_f32 = y_f32 ? 1 : 0;
+  g.acc_out = acc_out;
+  g.absmax = absmax;
+  g.w_scale = w_scale;
+  constexpr size_t smem = bl::gemm_sp2_smem_bytes();
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(bl::kSpThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters = -1;
+  if (max_clusters < 0) {
+    cudaError_t e = cudaFuncSetAttribute(bl::gemm_sp2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(sparse gemm)");
+    cfg.gridDim = dim3(2 * (device_sm_count() / 2));
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, bl::gemm_sp2_kernel, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(sparse gemm)");
+    max_clusters = n;
+  }
+  if (max_clusters <= 0) return fail(BL_ERR_CUDA, "no CTA pair of the sparse product fits on this device");
+  const int tiles = g.num_row_blocks * g.num_tok_blocks;
+  const int clusters = tiles < max_clusters ? tiles : max_clusters;
+  cfg.gridDim = dim3(2 * clusters);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, bl::gemm_sp2_kernel, ta, tb, te, ty, g);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse gemm launch");
+  return BL_OK;
 }
 
 inline size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
@@ -447,23 +589,29 @@ size_t bitlinear_quant_mask_workspace_size(int64_t n_out, int64_t k_in) {
 }
 
 bl_status bitlinear_quant_mask(const float* w_latent, int64_t n_out, int64_t k_in, int n_keep, int m_group,
-                               uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out, float* w_scale_out,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+                               uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out, int8_t* sp_values_out,
+                               uint8_t* sp_meta_out, float* w_scale_out, void* workspace, size_t workspace_bytes,
+                               void* stream) {
   g_err[0] = 0;
   if (!w_latent || !codes_out || !w_scale_out) return fail(BL_ERR_INVALID_ARG, "w_latent, codes_out, w_scale_out are required");
   if (bl_status s = check_shape(0, k_in, n_out)) return s;
   if (!(m_group == 4 || m_group == 8) || n_keep < 1 || n_keep > m_group)
     return fail(BL_ERR_INVALID_ARG, "N:M = %d:%d: need M in {4, 8} and 1 <= N <= M", n_keep, m_group);
+  if ((sp_values_out == nullptr) != (sp_meta_out == nullptr))
+    return fail(BL_ERR_INVALID_ARG, "give both sp_values_out and sp_meta_out, or neither");
+  if (sp_values_out && n_keep > 2)
+    return fail(BL_ERR_INVALID_ARG, "N:M = %d:%d is not 2:4-valid (at most 2 kept per aligned 4): no 2:4 storage",
+                n_keep, m_group);
   if (!workspace) return fail(BL_ERR_WORKSPACE, "workspace is required");
-  const int64_t numel = n_out * k_in;
   if (workspace_bytes < bitlinear_quant_mask_workspace_size(n_out, k_in))
     return fail(BL_ERR_WORKSPACE, "workspace too small: %zu < %zu", workspace_bytes,
                 bitlinear_quant_mask_workspace_size(n_out, k_in));
   if (!aligned16(w_latent) || !aligned16(codes_out) || !aligned16(w_scale_out) || !aligned16(workspace) ||
-      (mask_out && !aligned16(mask_out)) || (w_i8_out && !aligned16(w_i8_out)))
+      (mask_out && !aligned16(mask_out)) || (w_i8_out && !aligned16(w_i8_out)) ||
+      (sp_values_out && !aligned16(sp_values_out)) || (sp_meta_out && !aligned16(sp_meta_out)))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
-  return enqueue_quant_mask(w_latent, n_out, k_in, n_keep, m_group, mask_out, codes_out, w_i8_out, w_scale_out,
-                            workspace, as_stream(stream));
+  const QmOutputs o{mask_out, codes_out, w_i8_out, sp_values_out, sp_meta_out, k_in / 8, sp_meta_pitch(k_in)};
+  return enqueue_quant_mask(w_latent, n_out, k_in, n_keep, m_group, o, w_scale_out, workspace, as_stream(stream));
 }
 
 bl_status bitlinear_quant_mask_status(const void* workspace, void* stream) {
@@ -489,20 +637,25 @@ bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t
 }
 
 bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* codes, const int8_t* w_i8,
-                        const float* w_scale, int64_t t, int64_t k_in, int64_t n_out, int32_t* acc_out, void* y_out,
-                        int y_dtype, void* stream) {
+                        const int8_t* sp_values, const uint8_t* sp_meta, const float* w_scale, int64_t t, int64_t k_in,
+                        int64_t n_out, int32_t* acc_out, void* y_out, int y_dtype, void* stream) {
   g_err[0] = 0;
   if (!w_scale) return fail(BL_ERR_INVALID_ARG, "w_scale is required");
-  if (!codes && !w_i8) return fail(BL_ERR_INVALID_ARG, "give codes or w_i8");
+  if ((sp_values == nullptr) != (sp_meta == nullptr))
+    return fail(BL_ERR_INVALID_ARG, "give both sp_values and sp_meta, or neither");
+  if (!codes && !w_i8 && !sp_values) return fail(BL_ERR_INVALID_ARG, "give codes, w_i8 or sp_values + sp_meta");
   if (y_dtype != BL_OUT_BF16 && y_dtype != BL_OUT_F32) return fail(BL_ERR_INVALID_ARG, "y_dtype must be BL_OUT_BF16 or BL_OUT_F32");
   if (bl_status s = check_shape(t, k_in, n_out)) return s;
-  if (!aligned16(w_scale) || (codes && !aligned16(codes)) || (w_i8 && !aligned16(w_i8)))
+  if (!aligned16(w_scale) || (codes && !aligned16(codes)) || (w_i8 && !aligned16(w_i8)) ||
+      (sp_values && !aligned16(sp_values)) || (sp_meta && !aligned16(sp_meta)))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
   if (t == 0) return BL_OK;   // empty batch: the t-sized arrays may be NULL
   if (!xq || !absmax || !y_out) return fail(BL_ERR_INVALID_ARG, "xq, absmax, y_out are required");
   if (!aligned16(xq) || !aligned16(absmax) || !aligned16(y_out) || (acc_out && !aligned16(acc_out)))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
   cudaStream_t st = as_stream(stream);
+  if (sp_values)
+    return enqueue_fwd_sp(xq, absmax, sp_values, sp_meta, w_scale, t, k_in, n_out, acc_out, y_out, y_dtype == BL_OUT_F32, st);
   if (w_i8) return enqueue_fwd_i8(xq, absmax, w_i8, w_scale, t, k_in, n_out, acc_out, y_out, y_dtype == BL_OUT_F32, st);
   bl_fwd_problem prob{xq, absmax, codes, w_scale, t, k_in, n_out, acc_out, y_out};
   return launch_fwd_codes(&prob, 1, y_dtype == BL_OUT_F32, st);
@@ -587,6 +740,7 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const int8_t* xq,
     g.out = grad_x;
     g.out_f32 = 0;
     g.w_scale = w_scale;
+    set_raster(g, 2.0 * double(t) * double(n_out), 2.0 * double(n_out) * double(k_in));
     CUtensorMap to;
     if (bl_status s = make_out_map(&to, grad_x, t, k_in, false)) return s;
     bool launched = false;
@@ -625,6 +779,7 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const int8_t* xq,
     g.num_n_blocks = static_cast<int>((k_in + bl::kBN - 1) / bl::kBN);
     g.out = grad_w;
     g.out_f32 = grad_w_dtype == BL_OUT_F32;
+    set_raster(g, 2.0 * double(n_out) * double(t), 2.0 * double(t) * double(k_in));
     CUtensorMap to;
     if (bl_status s = make_out_map(&to, grad_w, n_out, k_in, g.out_f32)) return s;
     bool launched = false;
@@ -776,6 +931,6 @@ extern "C" bl_status bitlinear_quant_mask_noalloc(const float* w_latent, int64_t
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
   void* scratch = nullptr;
   if (bl_status s = noalloc_scratch(&scratch)) return s;
-  return enqueue_quant_mask(w_latent, n_out, k_in, n_keep, m_group, mask_out, codes_out, w_i8_out, w_scale_out, scratch,
-                            as_stream(stream));
+  const QmOutputs o{mask_out, codes_out, w_i8_out, nullptr, nullptr, k_in / 8, k_in / 8};
+  return enqueue_quant_mask(w_latent, n_out, k_in, n_keep, m_group, o, w_scale_out, scratch, as_stream(stream));
 }

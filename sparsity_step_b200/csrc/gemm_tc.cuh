@@ -52,12 +52,26 @@ struct GemmArgs {
   int M, N;                  // output [M, N], row-major, ld = N
   int num_k_blocks;          // ceil(K * elem_bytes / 128)
   int num_m_blocks, num_n_blocks;
+  int m_fastest;             // tile order: 1 = m blocks fastest (A re-read from L2), 0 = n blocks fastest
+  int a_l2, b_l2;            // L2 policy of the A / B loads (L2_NORMAL, L2_EVICT_FIRST, ...)
   void* out;                 // bf16 or f32
   int out_f32;
   int32_t* acc_out;          // EPI_FWD only, nullable
   const float* row_absmax;   // EPI_FWD: a_t per output row
   const float* w_scale;      // gamma (EPI_FWD, EPI_GRADX)
 };
+
+// Tile index -> (m block, n block) in the launch's raster order: the operand whose
+// blocks vary fastest is re-read across the tiles of a wave and should stay in L2.
+__device__ __forceinline__ void tile_coords(const GemmArgs& g, int tile, int& mb, int& nb) {
+  if (g.m_fastest) {
+    mb = tile % g.num_m_blocks;
+    nb = tile / g.num_m_blocks;
+  } else {
+    mb = tile / g.num_n_blocks;
+    nb = tile % g.num_n_blocks;
+  }
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -219,10 +233,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t ph = 0;
       long long issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile / g.num_n_blocks) * kBM;
-        const int n0 = (tile % g.num_n_blocks) * kBN;
-        for (int kb = 0; kb < g.num_k_blocks; ++kb) {
+      const uint64_t pa = l2_policy(g.a_l2), pb = l2_policy(g.b_l2);
+      int local = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+        int mb, nb;
+        tile_coords(g, tile, mb, nb);
+        const int m0 = mb * kBM;
+        const int n0 = nb * kBN;
+        for (int kq = 0; kq < g.num_k_blocks; ++kq) {
+          const int kb = (local & 1) ? g.num_k_blocks - 1 - kq : kq;   // serpentine K order
           if (!mbar_wait(empty0 + 8u * s, ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -232,16 +251,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t a_dst = sA + s * kABytes, b_dst = sB + s * kBBytes;
           const int kc = kI8 ? kb * 128 : kb * 64;   // K coordinate in elements (128 B per stage)
           if (kAMN) {
-            tma_load_2d(a_dst, &tmA, fb, m0, kc);
-            tma_load_2d(a_dst + 8192, &tmA, fb, m0 + 64, kc);
+            tma_load_2d_hint(a_dst, &tmA, fb, m0, kc, pa);
+            tma_load_2d_hint(a_dst + 8192, &tmA, fb, m0 + 64, kc, pa);
           } else {
-            tma_load_2d(a_dst, &tmA, fb, kc, m0);
+            tma_load_2d_hint(a_dst, &tmA, fb, kc, m0, pa);
           }
           if (kBMN) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + 8192 * j, &tmB, fb, n0 + 64 * j, kc);
+            for (int j = 0; j < 4; ++j) tma_load_2d_hint(b_dst + 8192 * j, &tmB, fb, n0 + 64 * j, kc, pb);
           } else {
-            tma_load_2d(b_dst, &tmB, fb, kc, n0);
+            tma_load_2d_hint(b_dst, &tmB, fb, kc, n0, pb);
           }
           ++issued;
           if (++s == kStages) {
@@ -328,8 +347,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int buf = local & 1;
       const uint32_t tph = static_cast<uint32_t>(local >> 1) & 1u;
       // the row scale does not depend on the accumulator: fetch it before waiting
-      const int row = (tile / g.num_n_blocks) * kBM + row_in_tile;
-      const int n0 = (tile % g.num_n_blocks) * kBN;
+      int mb, nb;
+      tile_coords(g, tile, mb, nb);
+      const int row = mb * kBM + row_in_tile;
+      const int n0 = nb * kBN;
       const bool row_ok = row < g.M;
       float rs = 1.0f;
       if (kEpi == EPI_FWD) {

@@ -60,6 +60,15 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
       : "memory");
 }
+// Same, with an L2 eviction policy for the loaded lines.
+__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                      int c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols) : "memory");
 }
@@ -158,10 +167,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t ph = 0;
       long long issued = 0;
       bool ok = true;
-      for (int tile = cluster; tile < num_tiles && ok; tile += nclusters) {
-        const int m0 = (tile / g.num_n_blocks) * 256 + 128 * static_cast<int>(rank);
-        const int n0 = (tile % g.num_n_blocks) * 256 + 128 * static_cast<int>(rank);
-        for (int kb = 0; kb < g.num_k_blocks; ++kb) {
+      const uint64_t pa = l2_policy(g.a_l2), pb = l2_policy(g.b_l2);
+      int local = 0;
+      for (int tile = cluster; tile < num_tiles && ok; tile += nclusters, ++local) {
+        int mb, nb;
+        tile_coords(g, tile, mb, nb);
+        const int m0 = mb * 256 + 128 * static_cast<int>(rank);
+        const int n0 = nb * 256 + 128 * static_cast<int>(rank);
+        for (int kq = 0; kq < g.num_k_blocks; ++kq) {
+          const int kb = (local & 1) ? g.num_k_blocks - 1 - kq : kq;   // serpentine K order
           if (!mbar_wait(empty0 + 8u * s, ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -171,16 +185,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t a_dst = sA + s * kAHalfBytes, b_dst = sB + s * kBHalfBytes;
           const int kc = kI8 ? kb * 128 : kb * 64;
           if (kAMN) {
-            tma_load_2d_pair(a_dst, &tmA, fb, m0, kc);
-            tma_load_2d_pair(a_dst + 8192, &tmA, fb, m0 + 64, kc);
+            tma_load_2d_pair_hint(a_dst, &tmA, fb, m0, kc, pa);
+            tma_load_2d_pair_hint(a_dst + 8192, &tmA, fb, m0 + 64, kc, pa);
           } else {
-            tma_load_2d_pair(a_dst, &tmA, fb, kc, m0);
+            tma_load_2d_pair_hint(a_dst, &tmA, fb, kc, m0, pa);
           }
           if (kBMN) {
-            tma_load_2d_pair(b_dst, &tmB, fb, n0, kc);
-            tma_load_2d_pair(b_dst + 8192, &tmB, fb, n0 + 64, kc);
+            tma_load_2d_pair_hint(b_dst, &tmB, fb, n0, kc, pb);
+            tma_load_2d_pair_hint(b_dst + 8192, &tmB, fb, n0 + 64, kc, pb);
           } else {
-            tma_load_2d_pair(b_dst, &tmB, fb, kc, n0);
+            tma_load_2d_pair_hint(b_dst, &tmB, fb, kc, n0, pb);
           }
           ++issued;
           if (++s == kStages2) {
@@ -264,8 +278,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int tile = cluster; tile < num_tiles; tile += nclusters, ++local) {
       const int buf = local & 1;
       const uint32_t tph = static_cast<uint32_t>(local >> 1) & 1u;
-      const int row = (tile / g.num_n_blocks) * 256 + row_in_tile;
-      const int n0 = (tile % g.num_n_blocks) * kBN;
+      int mb, nb;
+      tile_coords(g, tile, mb, nb);
+      const int row = mb * 256 + row_in_tile;
+      const int n0 = nb * kBN;
       const bool row_ok = row < g.M;
       float rs = 1.0f;
       if (kEpi == EPI_FWD) {

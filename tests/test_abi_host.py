@@ -38,18 +38,23 @@ def test_quant_mask_validation(L):
     ws = L.bitlinear_quant_mask_workspace_size(896, 896)
     assert ws >= 256 + 16
     # null latent weights
-    assert L.bitlinear_quant_mask(None, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -1
+    assert L.bitlinear_quant_mask(None, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -1
     # bad N:M
     for n, m in [(0, 8), (9, 8), (2, 3), (6, 16)]:
-        assert L.bitlinear_quant_mask(GOOD, 896, 896, n, m, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -1
+        assert L.bitlinear_quant_mask(GOOD, 896, 896, n, m, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -1
     # unsupported shapes
-    assert L.bitlinear_quant_mask(GOOD, 896, 900, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -2
-    assert L.bitlinear_quant_mask(GOOD, 8, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -2
+    assert L.bitlinear_quant_mask(GOOD, 896, 900, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -2
+    assert L.bitlinear_quant_mask(GOOD, 8, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -2
     # workspace
-    assert L.bitlinear_quant_mask(GOOD, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, None, ws, None) == -7
-    assert L.bitlinear_quant_mask(GOOD, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws - 1, None) == -7
+    assert L.bitlinear_quant_mask(GOOD, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, None, ws, None) == -7
+    assert L.bitlinear_quant_mask(GOOD, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws - 1, None) == -7
+    # the 2:4 outputs: both or neither, and only for masks with at most two kept per four
+    assert L.bitlinear_quant_mask(GOOD, 896, 896, 2, 4, GOOD, GOOD, GOOD, GOOD, None, GOOD, GOOD, ws, None) == -1
+    assert L.bitlinear_quant_mask(GOOD, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -1
+    assert "2:4" in _err(L)
+    assert L.bitlinear_quant_mask(GOOD, 896, 896, 2, 8, GOOD, GOOD, GOOD, BAD, GOOD, GOOD, GOOD, ws, None) == -3
     # alignment
-    assert L.bitlinear_quant_mask(BAD, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -3
+    assert L.bitlinear_quant_mask(BAD, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -3
     assert "aligned" in _err(L)
 
 
@@ -74,11 +79,16 @@ def test_act_quant_validation(L):
 
 def test_fwd_validation(L):
     args = dict(xq=GOOD, a=GOOD, codes=GOOD, wi8=GOOD, g=GOOD)
-    assert L.bitlinear_fwd(GOOD, GOOD, None, None, GOOD, 4, 896, 896, None, GOOD, 0, None) == -1
-    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, GOOD, 4, 896, 896, None, GOOD, 7, None) == -1
-    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, GOOD, 4, 896, 100, None, GOOD, 0, None) == -2
-    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, GOOD, 4, 896, 896, BAD, GOOD, 0, None) == -3
-    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, GOOD, 0, 896, 896, None, GOOD, 0, None) == 0
+    #                      xq    absmax codes w_i8  spv   spm   w_scale t  k_in n_out acc  y   dtype stream
+    assert L.bitlinear_fwd(GOOD, GOOD, None, None, None, None, GOOD, 4, 896, 896, None, GOOD, 0, None) == -1
+    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, None, None, GOOD, 4, 896, 896, None, GOOD, 7, None) == -1
+    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, None, None, GOOD, 4, 896, 100, None, GOOD, 0, None) == -2
+    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, None, None, GOOD, 4, 896, 896, BAD, GOOD, 0, None) == -3
+    assert L.bitlinear_fwd(GOOD, GOOD, GOOD, GOOD, None, None, GOOD, 0, 896, 896, None, GOOD, 0, None) == 0
+    # the 2:4 operand: both parts or neither, 16-byte aligned
+    assert L.bitlinear_fwd(GOOD, GOOD, None, None, GOOD, None, GOOD, 4, 896, 896, None, GOOD, 0, None) == -1
+    assert L.bitlinear_fwd(GOOD, GOOD, None, None, GOOD, BAD, GOOD, 4, 896, 896, None, GOOD, 0, None) == -3
+    assert L.bitlinear_fwd(GOOD, GOOD, None, None, GOOD, GOOD, GOOD, 0, 896, 896, None, GOOD, 0, None) == 0
     del args
 
 

@@ -79,6 +79,16 @@ def test_hand_act_quant_and_acc():
 
 # ----------------------------------------------------------------------- ties and operation order
 
+def test_hand_dequant_x_bf16():
+    q = np.array([[int(t) for t in G["deq_q"]]], dtype=np.int8)
+    a = np.array([float(G["deq_a"][0])], dtype=np.float32)
+    got = O.dequant_x_bf16(q, a)
+    assert got.ravel().tolist() == [float(t) for t in G["deq_x_bf16"]]
+    # the bf16 operand is within half a bf16 step of the exact value it rounds
+    exact = O.dequant_x(q, a)
+    assert np.all(np.abs(got - exact) <= np.abs(exact) * 2.0 ** -8)
+
+
 def test_hand_ternary_ties_round_to_even():
     """w/gamma exactly +-0.5 gives code 0 (ties to even), one ulp more gives 1, 1.5 clips."""
     g = np.float32(float(G["tie_gamma"][0]))

@@ -7,8 +7,8 @@ import torch
 
 import sparsity_step_b200 as B
 from oracle import bitlinear_oracle as O
-from parity_util import (assert_bf16_within_ulp, assert_exact, assert_f32_close, assert_grad_close, bf16_dev_to_bits,
-                         bits_to_dev_bf16, f32_to_dev, layer_inputs, sample_rows)
+from parity_util import (assert_bf16_within_ulp, assert_exact, assert_f32_close, assert_grad_close, bf16_bits_to_f64,
+                         bf16_dev_to_bits, bits_to_dev_bf16, f32_to_dev, layer_inputs, sample_rows)
 from sparsity_step_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -17,18 +17,30 @@ pytestmark = pytest.mark.gpu
 
 
 def gpu_quant_mask(w_np, n, m):
-    out = B.bitlinear_quant_mask(f32_to_dev(w_np), n, m)
+    # masks with at most two kept per aligned four also get their 2:4 form
+    out = B.bitlinear_quant_mask(f32_to_dev(w_np), n, m, want_sp=n <= 2)
     torch.cuda.synchronize()
     assert B.bitlinear_quant_mask_status(out["workspace"]) == 0
     return out
 
 
-def check_quant_mask(out, ref, tag):
+def check_quant_mask(out, ref, tag, sp_rows=None):
     g = out["w_scale"].cpu().numpy()[:1]
     assert_exact(g.view(np.uint32), np.array([ref["gamma"]], np.float32).view(np.uint32), f"{tag} gamma")
     assert_exact(out["mask"].cpu().numpy(), ref["mask"], f"{tag} mask")
     assert_exact(out["codes"].cpu().numpy(), ref["codes_packed"], f"{tag} codes")
     assert_exact(out["w_i8"].cpu().numpy(), ref["mcode"], f"{tag} w_i8")
+    if "sp_values" in out:
+        # the oracle's 2:4 storage is pure-Python loops: sampled rows on large tensors
+        rows = np.arange(ref["mcode"].shape[0]) if sp_rows is None else sp_rows
+        want = O.compress_2_4(ref["mcode"][rows], ref["keep"][rows])
+        n_out, k_in = ref["mcode"].shape
+        meta = out["sp_meta"].cpu().numpy()
+        assert meta.shape == B.sp_meta_shape(n_out, k_in)
+        assert_exact(out["sp_values"].cpu().numpy()[rows], want["values"], f"{tag} 2:4 values")
+        assert_exact(meta[rows, :k_in // 8], want["meta"], f"{tag} 2:4 metadata")
+        # padding rows and columns: positions 0 and 1 in every group
+        assert np.all(meta[:, k_in // 8:] == 0x44) and np.all(meta[n_out:, :] == 0x44), f"{tag} metadata padding"
 
 
 def gpu_act_quant(x_bits):
@@ -46,7 +58,9 @@ def check_fwd(qm_dev, xq, a, ref_qm, ref_q, ref_a, tag, rows=None, paths=("w_i8"
     """Forward on both requested weight operands; compares acc (exact), bf16 and f32 y."""
     acc_ref, y_ref = O.fwd(ref_q, ref_a, ref_qm["mcode"], ref_qm["gamma"], rows=rows)
     for path in paths:
-        kw = {"w_i8": qm_dev["w_i8"]} if path == "w_i8" else {"codes": qm_dev["codes"]}
+        kw = ({"w_i8": qm_dev["w_i8"]} if path == "w_i8" else
+              {"sp_values": qm_dev["sp_values"], "sp_meta": qm_dev["sp_meta"]} if path == "sp" else
+              {"codes": qm_dev["codes"]})
         y, acc = B.bitlinear_fwd(xq, a, qm_dev["w_scale"], n_out=ref_qm["mcode"].shape[0], want_acc=True, **kw)
         torch.cuda.synchronize()
         acc_np = acc.cpu().numpy()
@@ -92,7 +106,7 @@ def full_layer(cfg, tensor, t, k_in, n_out, n, m, *, outliers=True, bwd=True, pa
     tag = f"cfg{cfg} t{tensor} [{t}x{k_in}->{n_out}] {n}:{m}"
     ref_qm = O.quant_mask(w, n, m)
     qm = gpu_quant_mask(w, n, m)
-    check_quant_mask(qm, ref_qm, tag)
+    check_quant_mask(qm, ref_qm, tag, sp_rows=sample_rows(n_out, tensor + 3) if sample else None)
     ref_q, ref_a = O.act_quant(x)
     xq, a = gpu_act_quant(x)
     check_act_quant(xq, a, ref_q, ref_a, tag)
@@ -127,7 +141,37 @@ QWEN15_MLP = [("gate", 1536, 8960), ("up", 1536, 8960), ("down", 8960, 1536)]
 @pytest.mark.parametrize("idx", range(3), ids=[s[0] for s in QWEN15_MLP])
 def test_config3_nm_sweep(idx, nm):
     _, k_in, n_out = QWEN15_MLP[idx]
-    full_layer(3, idx, 8192, k_in, n_out, nm[0], nm[1], outliers=False, bwd=False, paths=("w_i8",), sample=True)
+    # 2:4-valid masks also run on the sparse tensor cores
+    paths = ("w_i8", "sp") if nm[0] <= 2 else ("w_i8",)
+    full_layer(3, idx, 8192, k_in, n_out, nm[0], nm[1], outliers=False, bwd=False, paths=paths, sample=True)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (2, 8)], ids=lambda v: f"{v[0]}of{v[1]}")
+@pytest.mark.parametrize("idx", range(len(QWEN05)), ids=[s[0] for s in QWEN05])
+def test_config2_qwen05_linears_sparse_24(idx, nm):
+    """The Qwen2.5-0.5B linears at 4096 tokens on the sparse tensor cores (k/v: 128
+    weight rows, so the second CTA of every pair tile is past the output)."""
+    _, k_in, n_out = QWEN05[idx]
+    full_layer(2, 20 + idx, 4096, k_in, n_out, nm[0], nm[1], bwd=False, paths=("sp",), sample=True)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (2, 8), (1, 4), (1, 8)], ids=lambda v: f"{v[0]}of{v[1]}")
+@pytest.mark.parametrize("t,k_in,n_out", [(1, 128, 128), (100, 640, 896), (224, 896, 272), (225, 1536, 256),
+                                          (500, 384, 528), (449, 11008, 144)])
+def test_sparse_24_ragged(t, k_in, n_out, nm):
+    """Ragged tokens (tile of 224), K (stages of 256 logical: 640, 896, 384 end on half
+    or quarter stages), and weight rows (pair tiles of 256) on the sparse product."""
+    full_layer(1, 60 + t, t, k_in, n_out, nm[0], nm[1], bwd=False, paths=("sp", "w_i8"))
+
+
+def test_sparse_24_storage_matches_oracle_with_ties():
+    """2:4 storage of masks built on tied magnitudes and all-zero groups."""
+    rng = np.random.default_rng(11)
+    mag = rng.integers(0, 3, size=(48, 256)).astype(np.float32) * np.float32(0.01)
+    w = (mag * np.where(rng.random((48, 256)) < 0.5, -1, 1)).astype(np.float32)
+    w[0, :8] = 0.0
+    for n, m in [(2, 4), (2, 8), (1, 4), (1, 8)]:
+        check_quant_mask(gpu_quant_mask(w, n, m), O.quant_mask(w, n, m), f"ties {n}:{m}")
 
 
 QWEN3B_MLP = [("gate", 2048, 11008), ("up", 2048, 11008), ("down", 11008, 2048)]
@@ -286,11 +330,16 @@ def test_grad_w_dequantised_x(t, k_in, n_out, with_grad_x):
                              qm["w_scale"] if with_grad_x else None, want_grad_x=with_grad_x, xq=xq, absmax=a,
                              flags=B.BL_GRADW_DEQUANT_X)
     torch.cuda.synchronize()
+    # element by element against the library's stated operand (X_deq rounded to bf16),
+    # and normwise against the exact X_deq the pages' reading rounds
+    got = bf16_dev_to_bits(gw)
+    assert_grad_close(got, O.grad_w(dy, x, x_deq=O.dequant_x_bf16(ref_q, ref_a)), "grad_w (dequantised x, bf16)")
     ref = O.grad_w(dy, x, x_deq=O.dequant_x(ref_q, ref_a))
-    assert_grad_close(bf16_dev_to_bits(gw), ref, "grad_w (dequantised x)")
-    # the two readings of X really differ here (1% x20 outliers): the option is not a no-op
+    assert np.max(np.abs(bf16_bits_to_f64(got) - ref)) / np.max(np.abs(ref)) <= 2e-2
+    # the two readings of X really differ here (1% x20 outliers): element by element far
+    # beyond the tolerance, so the option is not a no-op
     raw = O.grad_w(dy, x)
-    assert np.max(np.abs(ref - raw)) / np.max(np.abs(raw)) > 2e-2
+    assert np.max(np.abs(ref - raw) / np.maximum(np.abs(raw), 1e-3 * np.max(np.abs(raw)))) > 0.1
     if with_grad_x:
         assert_grad_close(bf16_dev_to_bits(gx), O.grad_x(dy, ref_qm["mcode"], ref_qm["gamma"]), "grad_x (same call)")
 
@@ -305,8 +354,11 @@ def test_grad_w_dequantised_x_training_shape():
                             flags=B.BL_GRADW_DEQUANT_X)
     torch.cuda.synchronize()
     rows = sample_rows(n_out, 5)
+    got = bf16_dev_to_bits(gw)[rows]
+    assert_grad_close(got, O.grad_w(dy, x, rows=rows, x_deq=O.dequant_x_bf16(ref_q, ref_a)),
+                      "grad_w (dequantised x, bf16) training shape")
     ref = O.grad_w(dy, x, rows=rows, x_deq=O.dequant_x(ref_q, ref_a))
-    assert_grad_close(bf16_dev_to_bits(gw)[rows], ref, "grad_w (dequantised x) training shape")
+    assert np.max(np.abs(bf16_bits_to_f64(got) - ref)) / np.max(np.abs(ref)) <= 2e-2
 
 
 def test_range_error_reported():
