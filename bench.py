@@ -43,9 +43,10 @@ CFG_INDEX = 4   # the training-step workload's seed block
 # source has changed).
 TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum (1 pass) on the full-size
-    # grad_W launch (16384 x 2048 x 11008, CTA-pair kernel): 724,534,528 B read +
-    # 42,022,912 B written
-    "bwd_grad_w": {"sha": "e0f2f761070bdee5", "bytes": 766557440},
+    # grad_W launch (16384 x 2048 x 11008, CTA-pair kernel, raster by operand size,
+    # serpentine K): 640,313,856 B read + 41,900,800 B written (the 11008 -> 2048 launch:
+    # 640,384,000 + 42,234,368)
+    "bwd_grad_w": {"sha": "da1ce434dceb301b", "bytes": 682214656},
 }
 
 

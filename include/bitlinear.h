@@ -150,7 +150,9 @@ bl_status bitlinear_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t
  *
  *   xq [t, k_in] int8, absmax [t] fp32 (from bitlinear_act_quant).
  *   The masked weights, in one of three forms (give at least one; the first given
- *   in this order is used):
+ *   in this order is used, except that with both the 2:4 form and w_i8 the library
+ *   picks per shape: the sparse product from 100 GOP dense-equivalent (2*t*k_in*n_out)
+ *   up, where it measured faster, the dense one below):
  *     sp_values [n_out, k_in / 2] int8 + sp_meta [n_sp, k_sp / 8] uint8 (padded, see
  *       bitlinear_quant_mask): the 2:4 form from bitlinear_quant_mask (masks with at
  *       most two kept per aligned four). Runs on the sparse tensor cores

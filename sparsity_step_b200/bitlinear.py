@@ -165,7 +165,8 @@ def bitlinear_fwd(xq: torch.Tensor, absmax: torch.Tensor, w_scale: torch.Tensor,
     """y = (xq . masked_codes^T) * absmax/127 * gamma; returns (y, acc or None).
 
     Weight operand: the 2:4 form (``sp_values`` + ``sp_meta``, sparse tensor cores),
-    else ``w_i8`` (dense tensor cores), else ``codes`` (2-bit codes decoded on chip)."""
+    else ``w_i8`` (dense tensor cores), else ``codes`` (2-bit codes decoded on chip).
+    With both the 2:4 form and ``w_i8`` the library picks per shape."""
     t, k_in = xq.shape
     dev = xq.device
     _need(xq, torch.int8, None, "xq")

@@ -161,15 +161,14 @@ inline bool use_cta_pair(int64_t m) { return m > bl::kBM; }
 // Raster order of one product. By default tiles walk n blocks fastest (every wave
 // re-reads all of B). When B is larger than L2 and A is small enough to stay there, m
 // blocks go fastest instead, so that A is re-read from L2 and B streams once (grad_W of
-// the down projection: X [16384 x 11008] bf16 is 360 MB; measured 1.91 -> 0.72 GB of
-// DRAM reads per launch). No eviction hints: marking the streamed operand evict-first
-// doubled the DRAM reads (its lines left L2 before the other tiles of the same wave
-// read them).
+// the down projection: X [16384 x 11008] bf16 is 360 MB; measured 1.91 -> 0.64 GB of
+// DRAM reads per launch with the serpentine K order of the kernels). Eviction hints on
+// the loads were measured and dropped: evict-first on the streamed operand doubled the
+// DRAM reads (its lines left L2 before the other tiles of the same wave read them), and
+// the hinted TMA form cost ~2 % of forward time.
 void set_raster(bl::GemmArgs& g, double a_bytes, double b_bytes) {
   constexpr double kL2Bytes = 96e6;   // usable share of the 126 MB L2
   g.m_fastest = (b_bytes > kL2Bytes && a_bytes < b_bytes && a_bytes <= 0.7 * kL2Bytes) ? 1 : 0;
-  g.a_l2 = bl::L2_NORMAL;
-  g.b_l2 = bl::L2_NORMAL;
 }
 
 // ------------------------------------------------------------------ grouped codes product
@@ -573,6 +572,17 @@ bl_status enqueue_fwd_sp(const int8_t* xq, const float* absmax, const int8_t* sp
   return BL_OK;
 }
 
+// Choice between the 2:4 sparse and the dense int8 product when the caller gives both
+// forms, from the measured crossover (forward per shape on B200): the sparse product wins
+// on the Qwen2.5-1.5B MLP products at 8192 tokens (225 GOP dense-equivalent each:
+// 1.07-1.32x) and loses on the Qwen2.5-0.5B products at 4096 tokens (up to 36 GOP:
+// 0.84-0.93x), where the fixed cost per tile (metadata copy, accumulator hand-off,
+// transposed epilogue) is not amortised.
+constexpr double kSparseMinOps = 100e9;
+inline bool use_sparse_product(int64_t t, int64_t k_in, int64_t n_out) {
+  return 2.0 * double(t) * double(k_in) * double(n_out) >= kSparseMinOps;
+}
+
 inline size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
 
 }  // namespace
@@ -654,7 +664,7 @@ bl_status bitlinear_fwd(const int8_t* xq, const float* absmax, const uint8_t* co
   if (!aligned16(xq) || !aligned16(absmax) || !aligned16(y_out) || (acc_out && !aligned16(acc_out)))
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
   cudaStream_t st = as_stream(stream);
-  if (sp_values)
+  if (sp_values && (!w_i8 || use_sparse_product(t, k_in, n_out)))
     return enqueue_fwd_sp(xq, absmax, sp_values, sp_meta, w_scale, t, k_in, n_out, acc_out, y_out, y_dtype == BL_OUT_F32, st);
   if (w_i8) return enqueue_fwd_i8(xq, absmax, w_i8, w_scale, t, k_in, n_out, acc_out, y_out, y_dtype == BL_OUT_F32, st);
   bl_fwd_problem prob{xq, absmax, codes, w_scale, t, k_in, n_out, acc_out, y_out};

@@ -53,7 +53,6 @@ struct GemmArgs {
   int num_k_blocks;          // ceil(K * elem_bytes / 128)
   int num_m_blocks, num_n_blocks;
   int m_fastest;             // tile order: 1 = m blocks fastest (A re-read from L2), 0 = n blocks fastest
-  int a_l2, b_l2;            // L2 policy of the A / B loads (L2_NORMAL, L2_EVICT_FIRST, ...)
   void* out;                 // bf16 or f32
   int out_f32;
   int32_t* acc_out;          // EPI_FWD only, nullable
@@ -233,7 +232,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t ph = 0;
       long long issued = 0;
       bool ok = true;
-      const uint64_t pa = l2_policy(g.a_l2), pb = l2_policy(g.b_l2);
       int local = 0;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
         int mb, nb;
@@ -251,16 +249,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t a_dst = sA + s * kABytes, b_dst = sB + s * kBBytes;
           const int kc = kI8 ? kb * 128 : kb * 64;   // K coordinate in elements (128 B per stage)
           if (kAMN) {
-            tma_load_2d_hint(a_dst, &tmA, fb, m0, kc, pa);
-            tma_load_2d_hint(a_dst + 8192, &tmA, fb, m0 + 64, kc, pa);
+            tma_load_2d(a_dst, &tmA, fb, m0, kc);
+            tma_load_2d(a_dst + 8192, &tmA, fb, m0 + 64, kc);
           } else {
-            tma_load_2d_hint(a_dst, &tmA, fb, kc, m0, pa);
+            tma_load_2d(a_dst, &tmA, fb, kc, m0);
           }
           if (kBMN) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_2d_hint(b_dst + 8192 * j, &tmB, fb, n0 + 64 * j, kc, pb);
+            for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + 8192 * j, &tmB, fb, n0 + 64 * j, kc);
           } else {
-            tma_load_2d_hint(b_dst, &tmB, fb, kc, n0, pb);
+            tma_load_2d(b_dst, &tmB, fb, kc, n0);
           }
           ++issued;
           if (++s == kStages) {

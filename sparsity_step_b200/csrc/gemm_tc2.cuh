@@ -60,15 +60,6 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
       : "memory");
 }
-// Same, with an L2 eviction policy for the loaded lines.
-__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
-                                                      int c1, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "l"(policy)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols) : "memory");
 }
@@ -167,7 +158,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t ph = 0;
       long long issued = 0;
       bool ok = true;
-      const uint64_t pa = l2_policy(g.a_l2), pb = l2_policy(g.b_l2);
       int local = 0;
       for (int tile = cluster; tile < num_tiles && ok; tile += nclusters, ++local) {
         int mb, nb;
@@ -185,16 +175,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t a_dst = sA + s * kAHalfBytes, b_dst = sB + s * kBHalfBytes;
           const int kc = kI8 ? kb * 128 : kb * 64;
           if (kAMN) {
-            tma_load_2d_pair_hint(a_dst, &tmA, fb, m0, kc, pa);
-            tma_load_2d_pair_hint(a_dst + 8192, &tmA, fb, m0 + 64, kc, pa);
+            tma_load_2d_pair(a_dst, &tmA, fb, m0, kc);
+            tma_load_2d_pair(a_dst + 8192, &tmA, fb, m0 + 64, kc);
           } else {
-            tma_load_2d_pair_hint(a_dst, &tmA, fb, kc, m0, pa);
+            tma_load_2d_pair(a_dst, &tmA, fb, kc, m0);
           }
           if (kBMN) {
-            tma_load_2d_pair_hint(b_dst, &tmB, fb, n0, kc, pb);
-            tma_load_2d_pair_hint(b_dst + 8192, &tmB, fb, n0 + 64, kc, pb);
+            tma_load_2d_pair(b_dst, &tmB, fb, n0, kc);
+            tma_load_2d_pair(b_dst + 8192, &tmB, fb, n0 + 64, kc);
           } else {
-            tma_load_2d_pair_hint(b_dst, &tmB, fb, kc, n0, pb);
+            tma_load_2d_pair(b_dst, &tmB, fb, kc, n0);
           }
           ++issued;
           if (++s == kStages2) {

@@ -164,6 +164,26 @@ def test_sparse_24_ragged(t, k_in, n_out, nm):
     full_layer(1, 60 + t, t, k_in, n_out, nm[0], nm[1], bwd=False, paths=("sp", "w_i8"))
 
 
+@pytest.mark.parametrize("t,k_in,n_out", [(300, 896, 896), (8192, 1536, 8960)])
+def test_sparse_or_dense_picked_per_shape(t, k_in, n_out):
+    """With both the 2:4 form and the int8 weights, the library picks the product per
+    shape (dense below 100 GOP, sparse above); either way the accumulators are exact."""
+    w, x, _ = layer_inputs(3, 90 + n_out % 7, t, k_in, n_out, outliers=False)
+    ref_qm = O.quant_mask(w, 2, 4)
+    qm = gpu_quant_mask(w, 2, 4)
+    ref_q, ref_a = O.act_quant(x)
+    xq, a = gpu_act_quant(x)
+    rows = sample_rows(t, 3)
+    acc_ref, y_ref = O.fwd(ref_q, ref_a, ref_qm["mcode"], ref_qm["gamma"], rows=rows)
+    y, acc = B.bitlinear_fwd(xq, a, qm["w_scale"], w_i8=qm["w_i8"], sp_values=qm["sp_values"], sp_meta=qm["sp_meta"],
+                             want_acc=True)
+    y2, _ = B.bitlinear_fwd(xq, a, qm["w_scale"], w_i8=qm["w_i8"], sp_values=qm["sp_values"], sp_meta=qm["sp_meta"])
+    torch.cuda.synchronize()
+    assert_exact(acc.cpu().numpy()[rows], acc_ref, "acc (picked product)")
+    assert_bf16_within_ulp(bf16_dev_to_bits(y)[rows], y_ref, "y (picked product)")
+    assert_bf16_within_ulp(bf16_dev_to_bits(y2)[rows], y_ref, "y (picked product, TMA-store epilogue)")
+
+
 def test_sparse_24_storage_matches_oracle_with_ties():
     """2:4 storage of masks built on tied magnitudes and all-zero groups."""
     rng = np.random.default_rng(11)
