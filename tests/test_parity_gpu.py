@@ -224,7 +224,7 @@ def test_config5_decode_batches(idx, layer):
                   f32=(b == 8))
 
 
-@pytest.mark.parametrize("b", [1, 3, 8, 12, 16, 32, 128])
+@pytest.mark.parametrize("b", [1, 2, 3, 8, 12, 16, 32, 128])
 def test_config5_grouped_layer(b):
     """All seven linears of one layer in one grouped launch, mixed shapes."""
     probs, refs = [], []
