@@ -336,14 +336,6 @@ struct QmOutputs {
 inline int64_t sp_rows(int64_t n_out) { return (n_out + bl::kSpPad - 1) / bl::kSpPad * bl::kSpPad; }
 inline int64_t sp_meta_pitch(int64_t k_in) { return (k_in + bl::kSpPad - 1) / bl::kSpPad * bl::kSpPad / 8; }
 
-template <int M, int NK>
-void launch_mask_codes(const float* w, int64_t n8, int n_keep, const float* gamma, const QmOutputs& o, int grid,
-                       cudaStream_t st) {
-  bl::qm_mask_codes_kernel<M, NK><<<grid, bl::kQmThreads, 0, st>>>(
-      reinterpret_cast<const float4*>(w), n8, n_keep, gamma, o.mask, reinterpret_cast<uint16_t*>(o.codes),
-      reinterpret_cast<uint2*>(o.w_i8), reinterpret_cast<uint32_t*>(o.sp_values), o.sp_meta, o.k8, o.meta_pitch);
-}
-
 int qm_blocks(int64_t numel);
 int qm_blocks_launch(int64_t numel, int resident);
 
@@ -359,43 +351,82 @@ int resident_blocks(K kern, int* cache) {
   return *cache;
 }
 
-// Both passes of steps a1 + a2 on `scratch` (its first 16 bytes are cleared here). Both
-// grids are one wave of resident blocks (grid-stride loops): a partial second wave
+// Pass 2 for one compile-time N:M and mask source; the 2:4 form exists only for
+// 2:4-valid masks (at most two kept per aligned four), so only those instantiate it.
+template <int M, int NK, bool kMaskIn>
+void launch_codes(const uint4* w4, int64_t n8, int n_keep, float* gamma, const QmOutputs& o, cudaStream_t st) {
+  constexpr bool kSpOk = NK <= 2;
+  static int occ = 0, occ_sp = 0;   // per instantiation
+  auto grid = [&](int resident) {
+    const int64_t g = (n8 + bl::kQmThreads - 1) / bl::kQmThreads;
+    const int64_t cap = int64_t(device_sm_count()) * resident;
+    return static_cast<int>(g < cap ? g : cap);
+  };
+  uint16_t* codes = reinterpret_cast<uint16_t*>(o.codes);
+  uint2* w_i8 = reinterpret_cast<uint2*>(o.w_i8);
+  if (kSpOk && o.sp_values != nullptr) {
+    auto k = bl::qm_codes_kernel<M, NK, kMaskIn, kSpOk>;
+    k<<<grid(resident_blocks(k, &occ_sp)), bl::kQmThreads, 0, st>>>(w4, n8, n_keep, gamma, o.mask, codes, w_i8,
+                                                                     reinterpret_cast<uint32_t*>(o.sp_values),
+                                                                     o.sp_meta, o.k8, o.meta_pitch);
+  } else {
+    auto k = bl::qm_codes_kernel<M, NK, kMaskIn, false>;
+    k<<<grid(resident_blocks(k, &occ)), bl::kQmThreads, 0, st>>>(w4, n8, n_keep, gamma, o.mask, codes, w_i8, nullptr,
+                                                                  nullptr, o.k8, o.meta_pitch);
+  }
+}
+
+// Both passes for one compile-time N:M. With a mask output, pass 1 ranks the groups and
+// stores the keep bits there, and pass 2 reads them back; without one, pass 2 ranks.
+// Both grids are one wave of resident blocks (grid-stride loops): a partial second wave
 // would leave most SMs idle at the end of each pass.
+template <int M, int NK>
+void launch_quant_mask(const float* w, int64_t numel, int n_keep, const QmOutputs& o, const bl::QmScratch& q,
+                       float* gamma, cudaStream_t st) {
+  const uint4* w4 = reinterpret_cast<const uint4*>(w);
+  const int64_t n8 = numel / 8;
+  const int sms = device_sm_count();
+  static int occ1 = 0;   // per instantiation
+  if (o.mask != nullptr) {
+    auto k1 = bl::qm_sum_mask_kernel<M, NK, true>;
+    k1<<<qm_blocks_launch(numel, sms * resident_blocks(k1, &occ1)), bl::kQmThreads, 0, st>>>(w4, n8, numel, n_keep, q,
+                                                                                               gamma, o.mask);
+    launch_codes<M, NK, true>(w4, n8, n_keep, gamma, o, st);
+  } else {
+    auto k1 = bl::qm_sum_mask_kernel<8, 8, false>;
+    k1<<<qm_blocks_launch(numel, sms * resident_blocks(k1, &occ1)), bl::kQmThreads, 0, st>>>(w4, n8, numel, n_keep, q,
+                                                                                               gamma, nullptr);
+    launch_codes<M, NK, false>(w4, n8, n_keep, gamma, o, st);
+  }
+}
+
+// Both passes of steps a1 + a2 on `scratch` (its first 16 bytes are cleared here).
 bl_status enqueue_quant_mask(const float* w, int64_t n_out, int64_t k_in, int n_keep, int m_group, const QmOutputs& o,
                              float* gamma, void* scratch, cudaStream_t st) {
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   cudaError_t e = cudaMemsetAsync(ws, 0, 16, st);   // range flag, status, blocks-done ticket
   if (e != cudaSuccess) return cuda_fail(e, "scratch reset");
   const int64_t numel = n_out * k_in;
-  static int occ_sum = 0;
-  const int blocks = qm_blocks_launch(numel, device_sm_count() * resident_blocks(bl::qm_abs_sum_kernel, &occ_sum));
-  bl::QmScratch q{reinterpret_cast<unsigned int*>(ws), reinterpret_cast<int*>(ws + 4),
-                  reinterpret_cast<unsigned int*>(ws + 8), reinterpret_cast<unsigned long long*>(ws + bl::kQmWsHeader)};
-  bl::qm_abs_sum_kernel<<<blocks, bl::kQmThreads, 0, st>>>(reinterpret_cast<const float4*>(w), numel / 4, numel, q, gamma);
-  const int64_t n8 = numel / 8;
-  int64_t g2 = (n8 + bl::kQmThreads - 1) / bl::kQmThreads;
-  static int occ_mask = 0;   // the same for every instantiation in practice (38-40 registers)
-  const int64_t cap = int64_t(device_sm_count()) * resident_blocks(bl::qm_mask_codes_kernel<8, 6>, &occ_mask);
-  if (g2 > cap) g2 = cap;
-  const int grid = static_cast<int>(g2);
+  const bl::QmScratch q{reinterpret_cast<unsigned int*>(ws), reinterpret_cast<int*>(ws + 4),
+                        reinterpret_cast<unsigned int*>(ws + 8),
+                        reinterpret_cast<unsigned long long*>(ws + bl::kQmWsHeader)};
   if (m_group == 8) {
     switch (n_keep) {
-      case 8: launch_mask_codes<8, 8>(w, n8, n_keep, gamma, o, grid, st); break;
-      case 7: launch_mask_codes<8, 7>(w, n8, n_keep, gamma, o, grid, st); break;
-      case 6: launch_mask_codes<8, 6>(w, n8, n_keep, gamma, o, grid, st); break;
-      case 5: launch_mask_codes<8, 5>(w, n8, n_keep, gamma, o, grid, st); break;
-      case 4: launch_mask_codes<8, 4>(w, n8, n_keep, gamma, o, grid, st); break;
-      case 3: launch_mask_codes<8, 3>(w, n8, n_keep, gamma, o, grid, st); break;
-      case 2: launch_mask_codes<8, 2>(w, n8, n_keep, gamma, o, grid, st); break;
-      default: launch_mask_codes<8, 1>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 8: launch_quant_mask<8, 8>(w, numel, n_keep, o, q, gamma, st); break;
+      case 7: launch_quant_mask<8, 7>(w, numel, n_keep, o, q, gamma, st); break;
+      case 6: launch_quant_mask<8, 6>(w, numel, n_keep, o, q, gamma, st); break;
+      case 5: launch_quant_mask<8, 5>(w, numel, n_keep, o, q, gamma, st); break;
+      case 4: launch_quant_mask<8, 4>(w, numel, n_keep, o, q, gamma, st); break;
+      case 3: launch_quant_mask<8, 3>(w, numel, n_keep, o, q, gamma, st); break;
+      case 2: launch_quant_mask<8, 2>(w, numel, n_keep, o, q, gamma, st); break;
+      default: launch_quant_mask<8, 1>(w, numel, n_keep, o, q, gamma, st); break;
     }
   } else {
     switch (n_keep) {
-      case 4: launch_mask_codes<4, 4>(w, n8, n_keep, gamma, o, grid, st); break;
-      case 3: launch_mask_codes<4, 3>(w, n8, n_keep, gamma, o, grid, st); break;
-      case 2: launch_mask_codes<4, 2>(w, n8, n_keep, gamma, o, grid, st); break;
-      default: launch_mask_codes<4, 1>(w, n8, n_keep, gamma, o, grid, st); break;
+      case 4: launch_quant_mask<4, 4>(w, numel, n_keep, o, q, gamma, st); break;
+      case 3: launch_quant_mask<4, 3>(w, numel, n_keep, o, q, gamma, st); break;
+      case 2: launch_quant_mask<4, 2>(w, numel, n_keep, o, q, gamma, st); break;
+      default: launch_quant_mask<4, 1>(w, numel, n_keep, o, q, gamma, st); break;
     }
   }
   e = cudaGetLastError();

@@ -6,17 +6,20 @@
 // BitNet b1.58 2B4T article (lsdiaocha.cn), section 一: absmean quantisation to
 // {-1, 0, +1}; section 四: four ternary values packed per byte.
 //
-// Two launches, both HBM-bound:
-//   qm_abs_sum_kernel   : grid-stride read of W (four 16-byte loads in flight per
-//                         thread), per-block exact integer sum of floor(|w| * 2^32);
-//                         the last block adds the partials (128-bit), rounds
-//                         S / (n * 2^32) once to fp32 and writes gamma = mean + 1e-5.
-//   qm_mask_codes_kernel: one thread per 8 contiguous weights (two 16-byte loads,
-//                         a warp covers 1 KB contiguous), walking W in reverse so
-//                         that pass 1's last lines, still in L2, come first; top-N
-//                         mask by knock-out tournaments, ternary codes by integer
-//                         arithmetic on the bit patterns, 2-bit packing, optional
-//                         int8 weights and 2:4 form.
+// Two launches, both streaming W (one thread = 8 contiguous weights = one group of 8 or
+// two groups of 4; a warp covers 1 KB contiguous; two groups per thread in flight):
+//   qm_sum_mask_kernel : exact integer sum of floor(|w| * 2^32) per block; when the
+//                        caller wants the mask, also the top-N keep bits (knock-out
+//                        tournaments; the mask needs no gamma), stored to the mask
+//                        output. The last block adds the partials (128-bit), rounds
+//                        S / (n * 2^32) once to fp32 and writes gamma = mean + 1e-5.
+//   qm_codes_kernel    : walks W in reverse (pass 1's last lines, still in L2, first),
+//                        reads the keep bits back (or ranks the group itself when no
+//                        mask output is wanted), and writes the ternary codes (integer
+//                        arithmetic on the bit patterns), their 2-bit packing, the
+//                        optional int8 weights and the optional 2:4 form.
+// Ranking in pass 1 puts the ALU-heavy tournaments in the pass that is otherwise bound
+// by memory latency, and leaves pass 2 a short stream of loads, byte permutes and stores.
 #pragma once
 
 #include "common.cuh"
@@ -28,9 +31,7 @@ namespace bl {
 // The first 16 bytes must be zero when a call starts (the host clears them).
 constexpr size_t kQmWsHeader = 256;
 constexpr int kQmThreads = 256;
-constexpr int kQmUnroll = 4;                        // 16-byte loads in flight per thread
 constexpr int64_t kQmMaxElemsPerThread = 1 << 14;   // keeps a thread's u64 sum < 2^62
-constexpr float kAbsLimit = 65536.0f;              // |w| < 2^16 is summed exactly
 
 struct QmScratch {
   unsigned int* range_flag;
@@ -39,34 +40,45 @@ struct QmScratch {
   unsigned long long* partials;
 };
 
-// 16-byte read-only loads without L1 allocation (W is read once per pass).
-__device__ __forceinline__ float4 ld_nc_f4(const float4* p) {
-  float4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint4 ld_nc_u4(const float4* p) {
+
+// 16-byte read-only loads without L1 allocation (W is read once per pass); `ok` false
+// gives zeros without a load.
+__device__ __forceinline__ uint4 ld_nc_u4(const uint4* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
 }
-
-__device__ __forceinline__ void qm_accumulate(const float4& v, uint64_t& acc, bool& bad) {
-  const float e[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float a = fabsf(e[j]);
-    if (a < kAbsLimit) {
-      // a * 2^32 is exact (power-of-two scale, < 2^48); truncation toward zero is floor
-      acc += __float2ull_rz(a * 4294967296.0f);
-    } else {
-      bad = true;   // also catches NaN (the comparison is false)
-    }
+struct QmPair {   // the 8 weights of one thread step (bit patterns)
+  uint4 lo, hi;
+};
+__device__ __forceinline__ QmPair qm_load(const uint4* w4, int64_t g, bool ok) {
+  QmPair v{make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  if (ok) {
+    v.lo = ld_nc_u4(w4 + 2 * g);
+    v.hi = ld_nc_u4(w4 + 2 * g + 1);
   }
+  return v;
+}
+
+// floor(|w| * 2^32) of 8 weights into the thread's sum: |w| * 2^32 is exact (a power-of-
+// two scale, < 2^48 for |w| < 2^16) and truncation toward zero is the floor; the eight
+// terms are added as a tree (short dependency chains). Range: |w| >= 2^16, inf and NaN
+// are exactly the |w| patterns >= 0x47800000, i.e. those whose sum with 0x38800000
+// reaches bit 31 (no overflow below 2^31 + 0x38800000); `bad` collects bit 31 of those
+// sums, tested after the loop.
+__device__ __forceinline__ void qm_accumulate8(const uint32_t (&b)[8], uint64_t& acc, uint32_t& bad) {
+  uint64_t u[8];
+  uint32_t r = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t a = b[j] & 0x7fffffffu;
+    r |= a + 0x38800000u;
+    u[j] = __float2ull_rz(__uint_as_float(a) * 4294967296.0f);
+  }
+  bad |= r;
+  acc += ((u[0] + u[1]) + (u[2] + u[3])) + ((u[4] + u[5]) + (u[6] + u[7]));
 }
 
 __device__ float rn_f32_ratio_u128(uint64_t slo, uint64_t shi, int64_t numel);
@@ -93,56 +105,6 @@ __device__ __forceinline__ void block_sum_u128(uint64_t& lo, uint64_t& hi) {
     lo = blo;
     hi = bhi;
   }
-}
-
-// Pass 1: exact integer sum of floor(|w| * 2^32). Each block stores its partial; the
-// last block to finish (atomic ticket) adds all partials, rounds the mean once to
-// fp32, writes gamma = mean + 1e-5 (NaN and status BL_ERR_RANGE on a range error)
-// and clears the ticket and the flag for the next call.
-__global__ void __launch_bounds__(kQmThreads) qm_abs_sum_kernel(const float4* __restrict__ w4, int64_t n4, int64_t numel,
-                                                                 QmScratch ws, float* __restrict__ gamma_out) {
-  uint64_t acc = 0;
-  bool bad = false;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; i + (kQmUnroll - 1) * stride < n4; i += kQmUnroll * stride) {
-    float4 v[kQmUnroll];
-#pragma unroll
-    for (int u = 0; u < kQmUnroll; ++u) v[u] = ld_nc_f4(w4 + i + u * stride);
-#pragma unroll
-    for (int u = 0; u < kQmUnroll; ++u) qm_accumulate(v[u], acc, bad);
-  }
-  for (; i < n4; i += stride) qm_accumulate(ld_nc_f4(w4 + i), acc, bad);
-  if (bad) atomicOr(ws.range_flag, 1u);
-
-  uint64_t lo = acc, hi = 0;
-  block_sum_u128(lo, hi);
-  __shared__ bool s_last;
-  if (threadIdx.x == 0) {
-    ws.partials[2 * blockIdx.x] = lo;
-    ws.partials[2 * blockIdx.x + 1] = hi;
-    __threadfence();   // the partial is visible before the ticket is taken
-    s_last = atomicAdd(ws.done, 1u) == gridDim.x - 1;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  lo = 0;
-  hi = 0;
-  for (int b = threadIdx.x; b < static_cast<int>(gridDim.x); b += blockDim.x)
-    add_u128(lo, hi, __ldcg(ws.partials + 2 * b), __ldcg(ws.partials + 2 * b + 1));
-  block_sum_u128(lo, hi);
-  if (threadIdx.x != 0) return;
-  const unsigned int flag = atomicAdd(ws.range_flag, 0u);
-  *ws.range_flag = 0;   // leave the scratch ready for the next call
-  *ws.done = 0;
-  if (flag) {
-    *ws.status = -4;   // BL_ERR_RANGE
-    *gamma_out = __int_as_float(0x7fc00000);
-    return;
-  }
-  *ws.status = 0;
-  *gamma_out = __fadd_rn(rn_f32_ratio_u128(lo, hi, numel), 1e-5f);   // one fp32 add
 }
 
 // ---- exact rounding of S / D to fp32 (round to nearest, ties to even) ----------
@@ -206,16 +168,26 @@ __device__ float rn_f32_ratio_u128(uint64_t slo, uint64_t shi, int64_t numel) {
 }
 
 
-// ---- integer helpers of the mask/code pass (host-callable, so that host tests can
+// ---- integer helpers of the mask/code passes (host-callable, so that host tests can
 // check them against brute force) ---------------------------------------------------
 
+// Byte permute with the full PTX semantics: selector nibble bits 0-2 pick one of the
+// eight bytes of {y, x} (x = bytes 0-3), bit 3 replicates the picked byte's sign bit
+// over the result byte.
 __host__ __device__ __forceinline__ uint32_t qm_prmt(uint32_t x, uint32_t y, uint32_t sel) {
 #ifdef __CUDA_ARCH__
-  return __byte_perm(x, y, sel);
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(x), "r"(y), "r"(sel));
+  return r;
 #else
   const uint64_t v = (static_cast<uint64_t>(y) << 32) | x;
   uint32_t r = 0;
-  for (int k = 0; k < 4; ++k) r |= static_cast<uint32_t>((v >> (8 * ((sel >> (4 * k)) & 7u))) & 0xFFu) << (8 * k);
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t s = (sel >> (4 * k)) & 0xFu;
+    uint32_t byte = static_cast<uint32_t>((v >> (8 * (s & 7u))) & 0xFFu);
+    if (s & 8u) byte = (byte & 0x80u) ? 0xFFu : 0x00u;
+    r |= byte << (8 * k);
+  }
   return r;
 #endif
 }
@@ -355,17 +327,14 @@ __host__ __device__ __forceinline__ uint32_t group_keep(const uint32_t (&a)[8], 
 // on the bit patterns of non-negative floats the comparison is an unsigned compare.
 //
 // Four codes as int8 bytes (+1, -1, 0) of weights b[0..3] (bit patterns; a = |w|
-// patterns): m = -1 when |w| > gamma/2 (the sign of half - a, both below 2^31), s = -1
-// for negative w, code byte = low byte of m & (s | 1); three byte permutes gather them.
+// patterns): half - a is negative exactly when |w| > gamma/2 (both below 2^31); byte
+// permutes with sign replication turn the four sign bits of (half - a) into a byte mask
+// `mag` and the four sign bits of w into a byte mask `neg`; code = mag & (neg | 0x01).
 __host__ __device__ __forceinline__ uint32_t qm_code_word(const uint32_t* b, const uint32_t* a, uint32_t half_bits) {
-  uint32_t c[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t m = static_cast<uint32_t>(static_cast<int32_t>(half_bits - a[j]) >> 31);
-    const uint32_t sg = static_cast<uint32_t>(static_cast<int32_t>(b[j]) >> 31);
-    c[j] = m & (sg | 1u);
-  }
-  return qm_prmt(qm_prmt(c[0], c[1], 0x0040u), qm_prmt(c[2], c[3], 0x0040u), 0x5410u);
+  const uint32_t t0 = half_bits - a[0], t1 = half_bits - a[1], t2 = half_bits - a[2], t3 = half_bits - a[3];
+  const uint32_t mag = qm_prmt(qm_prmt(t0, t1, 0x00FBu), qm_prmt(t2, t3, 0xFB00u), 0x7610u);
+  const uint32_t neg = qm_prmt(qm_prmt(b[0], b[1], 0x00FBu), qm_prmt(b[2], b[3], 0xFB00u), 0x7610u);
+  return mag & (neg | 0x01010101u);
 }
 
 // Four keep bits -> a byte mask (0xFF for each kept byte): bit j moves to bit 8j
@@ -374,13 +343,15 @@ __host__ __device__ __forceinline__ uint32_t qm_keep_bytes(uint32_t k4) {
   return ((k4 * 0x00204081u) & 0x01010101u) * 0xFFu;
 }
 
-// int8 code word (bytes +1 / -1 / 0) -> its four 2-bit codes (01 / 11 / 00) in one byte,
-// element j at bits 2j.
-__host__ __device__ __forceinline__ uint32_t qm_pack2(uint32_t w) {
-  uint32_t x = w & 0x03030303u;
-  x |= x >> 6;
-  x |= x >> 12;
-  return x & 0xFFu;
+// Two int8 code words (bytes +1 / -1 / 0; lo = elements 0-3, hi = 4-7) -> their eight
+// 2-bit codes (01 / 11 / 00), element j at bits 2j. The low two bits of each byte are
+// the code; one multiply gathers the four fields of a word into its top byte (field k
+// moves from bit 8k to bit 24 + 2k; every other partial product lands below bit 24 in a
+// field of its own, so no carry reaches the top byte), and a byte permute joins the two.
+__host__ __device__ __forceinline__ uint32_t qm_pack16(uint32_t lo, uint32_t hi) {
+  const uint32_t x = (lo & 0x03030303u) * 0x01041040u;
+  const uint32_t y = (hi & 0x03030303u) * 0x01041040u;
+  return qm_prmt(x, y, 0x0073u) & 0xFFFFu;
 }
 
 // 2:4 storage of one group of four (keep nibble kb, at most two bits set): the two
@@ -395,46 +366,127 @@ __host__ __device__ __forceinline__ uint32_t sp24_nibble(uint32_t kb) {
   return i0 | (i1 << 2);
 }
 
-// Everything the mask/code pass derives from 8 contiguous weights (one group of 8, or
-// two groups of 4): the keep bits, the masked int8 codes (lo = elements 0-3, hi = 4-7),
-// the packed 2-bit codes, and the 2:4 form (values word and metadata byte).
-struct QmGroup8 {
-  uint32_t keep, lo, hi, packed, sp_values, sp_meta;
+// Keep bits of the thread's 8 weights (bit patterns b; |w| patterns are order-
+// preserving): one group of 8, or two groups of 4.
+template <int M, int NK>
+__host__ __device__ __forceinline__ uint32_t qm_keep8(const uint32_t (&b)[8], int n_keep) {
+  uint32_t a[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = b[j] & 0x7fffffffu;
+  uint32_t keep = group_keep<M, NK, 0>(a, n_keep);
+  if (M == 4) keep |= group_keep<M, NK, 4>(a, n_keep);
+  return keep;
+}
+
+// Everything pass 2 derives from 8 contiguous weights and their keep bits: the masked
+// int8 codes (lo = elements 0-3, hi = 4-7), the packed 2-bit codes, and the 2:4 form
+// (values word and metadata byte).
+struct QmCodes8 {
+  uint32_t lo, hi, packed, sp_values, sp_meta;
 };
 
-template <int M, int NK>
-__host__ __device__ __forceinline__ QmGroup8 qm_group8(const uint32_t (&b)[8], int n_keep, uint32_t half_gamma_bits,
+template <bool kSp>
+__host__ __device__ __forceinline__ QmCodes8 qm_codes8(const uint32_t (&b)[8], uint32_t keep, uint32_t half_gamma_bits,
                                                        bool gamma_ok) {
   uint32_t a[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) a[j] = b[j] & 0x7fffffffu;   // |w| bits: order-preserving
-  QmGroup8 r;
-  r.keep = group_keep<M, NK, 0>(a, n_keep);
-  if (M == 4) r.keep |= group_keep<M, NK, 4>(a, n_keep);
-  const uint32_t code_keep = gamma_ok ? r.keep : 0u;   // range error: all codes 0 (gamma is NaN)
+  for (int j = 0; j < 8; ++j) a[j] = b[j] & 0x7fffffffu;
+  QmCodes8 r;
+  const uint32_t code_keep = gamma_ok ? keep : 0u;   // range error: all codes 0 (gamma is NaN)
   r.lo = qm_code_word(b, a, half_gamma_bits) & qm_keep_bytes(code_keep & 0xFu);
   r.hi = qm_code_word(b + 4, a + 4, half_gamma_bits) & qm_keep_bytes(code_keep >> 4);
-  r.packed = qm_pack2(r.lo) | (qm_pack2(r.hi) << 8);
-  // 2:4 form (meaningful for masks with at most two kept per aligned four): masked
-  // codes are 0 at unkept positions, so one byte permute picks each group's two values
-  const uint32_t n0 = sp24_nibble(r.keep & 0xFu), n1 = sp24_nibble((r.keep >> 4) & 0xFu);
-  r.sp_values = qm_prmt(r.lo, r.hi, (n0 & 3u) | ((n0 >> 2) << 4) | ((4u + (n1 & 3u)) << 8) | ((4u + (n1 >> 2)) << 12));
-  r.sp_meta = n0 | (n1 << 4);
+  r.packed = qm_pack16(r.lo, r.hi);
+  r.sp_values = r.sp_meta = 0;
+  if (kSp) {
+    // 2:4 form (meaningful for masks with at most two kept per aligned four): masked
+    // codes are 0 at unkept positions, so one byte permute picks each group's two values
+    const uint32_t n0 = sp24_nibble(keep & 0xFu), n1 = sp24_nibble((keep >> 4) & 0xFu);
+    r.sp_values =
+        qm_prmt(r.lo, r.hi, (n0 & 3u) | ((n0 >> 2) << 4) | ((4u + (n1 & 3u)) << 8) | ((4u + (n1 >> 2)) << 12));
+    r.sp_meta = n0 | (n1 << 4);
+  }
   return r;
 }
 
-// Pass 2 of steps a1 + a2. One thread = 8 contiguous weights (one group of 8, or two
-// groups of 4). Walks W in reverse (grid-stride from the end) so that the lines pass 1
-// read last, still in L2, are read first (measured: 43 % of W from L2 for a 90 MB tensor).
-template <int M, int NK>
-__global__ void __launch_bounds__(kQmThreads) qm_mask_codes_kernel(const float4* __restrict__ w4, int64_t n8, int n_keep,
-                                                                    const float* __restrict__ gamma_ptr,
-                                                                    uint8_t* __restrict__ mask_out,
-                                                                    uint16_t* __restrict__ codes_out,
-                                                                    uint2* __restrict__ w_i8_out,
-                                                                    uint32_t* __restrict__ sp_values_out,
-                                                                    uint8_t* __restrict__ sp_meta_out, int64_t k8,
-                                                                    int64_t meta_pitch) {
+// Pass 1: exact integer sum of floor(|w| * 2^32) and, with kMask, the keep bits of
+// every group stored to `mask`. Each block stores its partial sum; the last block to
+// finish (atomic ticket) adds all partials, rounds the mean once to fp32, writes
+// gamma = mean + 1e-5 (NaN and status BL_ERR_RANGE on a range error) and clears the
+// ticket and the flag for the next call. Two thread steps are in flight per thread
+// (register double buffer; loads past the end give zeros, which add nothing).
+template <int M, int NK, bool kMask>
+__global__ void __launch_bounds__(kQmThreads) qm_sum_mask_kernel(const uint4* __restrict__ w4, int64_t n8,
+                                                                  int64_t numel, int n_keep, QmScratch ws,
+                                                                  float* __restrict__ gamma_out,
+                                                                  uint8_t* __restrict__ mask) {
+  static_assert(M == 4 || M == 8, "groups of 4 or 8");
+  uint64_t acc = 0;
+  uint32_t bad = 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  auto step = [&](const QmPair& v, int64_t g) {
+    const uint32_t b[8] = {v.lo.x, v.lo.y, v.lo.z, v.lo.w, v.hi.x, v.hi.y, v.hi.z, v.hi.w};
+    qm_accumulate8(b, acc, bad);
+    if (kMask) {
+      const uint32_t keep = qm_keep8<M, NK>(b, n_keep);
+      if (M == 8) mask[g] = static_cast<uint8_t>(keep);
+      else reinterpret_cast<uint16_t*>(mask)[g] = static_cast<uint16_t>((keep & 0xFu) | ((keep >> 4) << 8));
+    }
+  };
+  int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  QmPair va = qm_load(w4, g, g < n8), vb;
+  for (; g < n8; g += 2 * stride) {
+    vb = qm_load(w4, g + stride, g + stride < n8);
+    step(va, g);
+    if (g + stride >= n8) break;
+    va = qm_load(w4, g + 2 * stride, g + 2 * stride < n8);
+    step(vb, g + stride);
+  }
+  if (bad & 0x80000000u) atomicOr(ws.range_flag, 1u);   // |w| >= 2^16, inf or NaN
+
+  uint64_t lo = acc, hi = 0;
+  block_sum_u128(lo, hi);
+  __shared__ bool s_last;
+  if (threadIdx.x == 0) {
+    ws.partials[2 * blockIdx.x] = lo;
+    ws.partials[2 * blockIdx.x + 1] = hi;
+    __threadfence();   // the partial is visible before the ticket is taken
+    s_last = atomicAdd(ws.done, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  lo = 0;
+  hi = 0;
+  for (int b = threadIdx.x; b < static_cast<int>(gridDim.x); b += blockDim.x)
+    add_u128(lo, hi, __ldcg(ws.partials + 2 * b), __ldcg(ws.partials + 2 * b + 1));
+  block_sum_u128(lo, hi);
+  if (threadIdx.x != 0) return;
+  const unsigned int flag = atomicAdd(ws.range_flag, 0u);
+  *ws.range_flag = 0;   // leave the scratch ready for the next call
+  *ws.done = 0;
+  if (flag) {
+    *ws.status = -4;   // BL_ERR_RANGE
+    *gamma_out = __int_as_float(0x7fc00000);
+    return;
+  }
+  *ws.status = 0;
+  *gamma_out = __fadd_rn(rn_f32_ratio_u128(lo, hi, numel), 1e-5f);   // one fp32 add
+}
+
+// Pass 2 of steps a1 + a2. One thread = 8 contiguous weights. Walks W in reverse
+// (grid-stride from the end) so that the lines pass 1 read last, still in L2, are read
+// first. kMaskIn: the keep bits come from pass 1 through `mask`; otherwise (no mask
+// output wanted) they are ranked here and `mask` is unused. kSp: also the 2:4 form
+// (the host allows it only for 2:4-valid masks).
+template <int M, int NK, bool kMaskIn, bool kSp>
+__global__ void __launch_bounds__(kQmThreads) qm_codes_kernel(const uint4* __restrict__ w4, int64_t n8, int n_keep,
+                                                              const float* __restrict__ gamma_ptr,
+                                                              const uint8_t* __restrict__ mask,
+                                                              uint16_t* __restrict__ codes_out,
+                                                              uint2* __restrict__ w_i8_out,
+                                                              uint32_t* __restrict__ sp_values_out,
+                                                              uint8_t* __restrict__ sp_meta_out, int64_t k8,
+                                                              int64_t meta_pitch) {
   static_assert(M == 4 || M == 8, "groups of 4 or 8");
   const float gamma = *gamma_ptr;
   const bool gamma_ok = isfinite(gamma) && gamma > 0.0f;
@@ -444,36 +496,27 @@ __global__ void __launch_bounds__(kQmThreads) qm_mask_codes_kernel(const float4*
   // the padded metadata has a row pitch of meta_pitch bytes: track this thread's (row,
   // column) of the k8 bytes per row, stepping back by `stride` without dividing
   int64_t mrow = 0, mcol = 0, sq = 0, sr = 0;
-  if (sp_meta_out != nullptr && tid < n8) {
+  if (kSp && tid < n8) {
     mrow = (n8 - 1 - tid) / k8;
     mcol = (n8 - 1 - tid) % k8;
     sq = stride / k8;
     sr = stride % k8;
   }
-  // the next iteration's 32 bytes are loaded before this one is processed
-  uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
-  if (tid < n8) {
-    n0 = ld_nc_u4(w4 + 2 * (n8 - 1 - tid));
-    n1 = ld_nc_u4(w4 + 2 * (n8 - 1 - tid) + 1);
-  }
-  for (int64_t r = tid; r < n8; r += stride) {
-    const int64_t i = n8 - 1 - r;
-    const uint4 v0 = n0, v1 = n1;
-    if (r + stride < n8) {
-      n0 = ld_nc_u4(w4 + 2 * (i - stride));
-      n1 = ld_nc_u4(w4 + 2 * (i - stride) + 1);
-    }
-    const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    const QmGroup8 g = qm_group8<M, NK>(b, n_keep, half_gamma_bits, gamma_ok);
-    codes_out[i] = static_cast<uint16_t>(g.packed);
-    if (mask_out != nullptr) {
-      if (M == 8) mask_out[i] = static_cast<uint8_t>(g.keep);
-      else reinterpret_cast<uint16_t*>(mask_out)[i] = static_cast<uint16_t>((g.keep & 0xFu) | ((g.keep >> 4) << 8));
-    }
-    if (w_i8_out != nullptr) w_i8_out[i] = make_uint2(g.lo, g.hi);
-    if (sp_values_out != nullptr) {   // the host allows it only for 2:4-valid masks
-      sp_values_out[i] = g.sp_values;
-      sp_meta_out[mrow * meta_pitch + mcol] = static_cast<uint8_t>(g.sp_meta);
+  auto load_keep = [&](int64_t i, bool ok) -> uint32_t {
+    if (!kMaskIn || !ok) return 0u;
+    if (M == 8) return mask[i];
+    const uint32_t m2 = reinterpret_cast<const uint16_t*>(mask)[i];
+    return (m2 & 0xFu) | ((m2 >> 8) << 4);
+  };
+  auto step = [&](const QmPair& v, uint32_t keep, int64_t i) {
+    const uint32_t b[8] = {v.lo.x, v.lo.y, v.lo.z, v.lo.w, v.hi.x, v.hi.y, v.hi.z, v.hi.w};
+    if (!kMaskIn) keep = qm_keep8<M, NK>(b, n_keep);
+    const QmCodes8 c = qm_codes8<kSp>(b, keep, half_gamma_bits, gamma_ok);
+    codes_out[i] = static_cast<uint16_t>(c.packed);
+    if (w_i8_out != nullptr) w_i8_out[i] = make_uint2(c.lo, c.hi);
+    if (kSp) {
+      sp_values_out[i] = c.sp_values;
+      sp_meta_out[mrow * meta_pitch + mcol] = static_cast<uint8_t>(c.sp_meta);
       mcol -= sr;
       mrow -= sq;
       if (mcol < 0) {
@@ -481,6 +524,20 @@ __global__ void __launch_bounds__(kQmThreads) qm_mask_codes_kernel(const float4*
         mrow -= 1;
       }
     }
+  };
+  // thread step r covers group index i = n8 - 1 - r; two steps in flight per thread
+  int64_t r = tid;
+  QmPair va = qm_load(w4, n8 - 1 - r, r < n8), vb;
+  uint32_t ka = load_keep(n8 - 1 - r, r < n8), kb;
+  for (; r < n8; r += 2 * stride) {
+    const int64_t r1 = r + stride, r2 = r + 2 * stride;
+    vb = qm_load(w4, n8 - 1 - r1, r1 < n8);
+    kb = load_keep(n8 - 1 - r1, r1 < n8);
+    step(va, ka, n8 - 1 - r);
+    if (r1 >= n8) break;
+    va = qm_load(w4, n8 - 1 - r2, r2 < n8);
+    ka = load_keep(n8 - 1 - r2, r2 < n8);
+    step(vb, kb, n8 - 1 - r1);
   }
 }
 
