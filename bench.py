@@ -685,10 +685,17 @@ def run_case(args) -> None:
     ws_i8 = (torch.empty((B.bitlinear_grad_x_i8_workspace_size(t, k_in, n_out),), dtype=torch.uint8, device=dev)
              if args.case == "grad_x_i8" else None)
     hist = torch.empty((19,), dtype=torch.int64, device=dev)
+    g_w = (bf(synth.activation_bf16(14, n_out, k_in, std=1e-2, outliers=False)) if args.case == "sgd_quant_mask"
+           else None)
     flops = 2.0 * t * k_in * n_out
     cases = {
+        # algorithmic bytes: W read once (4 B/w), int8 codes, packed codes and mask written
         "quant_mask": (lambda: B.bitlinear_quant_mask(w, N_KEEP, M_GROUP, out=qm, workspace=qm["workspace"]),
-                       "GB/s", n_out * k_in * (4 + 4 + 1 + 0.25 + 0.125)),
+                       "GB/s", n_out * k_in * (4 + 1 + 0.25 + 1.0 / M_GROUP)),
+        # the same plus the fused SGD step: gradient read (2 B/w), W written back (4 B/w)
+        "sgd_quant_mask": (lambda: B.bitlinear_sgd_quant_mask(w, g_w, 1e-3, N_KEEP, M_GROUP, out=qm,
+                                                              workspace=qm["workspace"]),
+                           "GB/s", n_out * k_in * (4 + 2 + 4 + 1 + 0.25 + 1.0 / M_GROUP)),
         "act_quant": (lambda: B.bitlinear_act_quant(x, xq=xq, absmax=a), "GB/s", t * k_in * 3 + 4 * t),
         "fwd": (lambda: B.bitlinear_fwd(xq, a, qm["w_scale"], w_i8=qm["w_i8"], y=y), "TOP/s", flops),
         # 2:4 mask on the sparse tensor cores: dense-equivalent ops
@@ -944,7 +951,7 @@ def main(argv=None) -> None:
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the N:M sweep and decode sub-records")
-    ap.add_argument("--case", choices=["quant_mask", "act_quant", "fwd", "fwd_sp", "fwd_codes", "grad_x", "grad_w",
+    ap.add_argument("--case", choices=["quant_mask", "sgd_quant_mask", "act_quant", "fwd", "fwd_sp", "fwd_codes", "grad_x", "grad_w",
                                        "grad_x_i8", "mask_hist", "mma_peak_i8", "mma_peak_bf16", "mma_peak_sp_i8"],
                     help="time one kernel class alone on the --case-t/k/n shape")
     ap.add_argument("--case-t", type=int, default=TOKENS)

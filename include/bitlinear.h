@@ -105,6 +105,32 @@ bl_status bitlinear_quant_mask(const float* w_latent, int64_t n_out, int64_t k_i
                                uint8_t* sp_meta_out, float* w_scale_out, void* workspace, size_t workspace_bytes,
                                void* stream);
 
+/*
+ * The latent-weight update of a training step fused with steps a1 + a2: the mask and
+ * codes are recomputed every step from the weights the optimizer has just updated
+ * (Sparse-BitNet article, section 三), so the update and the mask recompute share one
+ * read of W instead of two. The pages name no optimizer; this is plain SGD:
+ *
+ *   W <- fp32(W - lr * G)     (G the bf16 gradient; one rounding per weight: a fused
+ *                              multiply-add, round to nearest even)
+ *
+ * then exactly bitlinear_quant_mask of the updated W (same outputs, layouts and rules).
+ *
+ *   w_latent  [n_out, k_in] fp32, in/out: updated in place.
+ *   grad_w    [n_out, k_in] bf16 (bit patterns), in. The gradient of W, e.g. grad_w
+ *             of bitlinear_bwd.
+ *   lr        finite fp32, else BL_ERR_INVALID_ARG.
+ *   other arguments: as bitlinear_quant_mask.
+ *
+ * A range error of the UPDATED weights is reported as in bitlinear_quant_mask (the
+ * update has then been applied). Calls that share a workspace must not overlap on the
+ * GPU; w_latent must not overlap any output.
+ */
+bl_status bitlinear_sgd_quant_mask(float* w_latent, const uint16_t* grad_w, float lr, int64_t n_out, int64_t k_in,
+                                   int n_keep, int m_group, uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out,
+                                   int8_t* sp_values_out, uint8_t* sp_meta_out, float* w_scale_out, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then returns the range status (BL_OK or BL_ERR_RANGE) that
  * the last bitlinear_quant_mask using `workspace` recorded. */
 bl_status bitlinear_quant_mask_status(const void* workspace, void* stream);

@@ -213,6 +213,49 @@ def quant_mask(w: np.ndarray, n_keep: int, m_group: int) -> dict:
     }
 
 
+# --------------------------------------------------------------------------- optimizer step + a1, a2
+
+def sgd_update(w: np.ndarray, g_bits: np.ndarray, lr: float) -> np.ndarray:
+    """W <- fp32(W - lr * G): the latent-weight update that precedes the mask recompute.
+
+    Follows: Sparse-BitNet article section 三 (the mask is recomputed at every training
+    step from the latent weights that step has just updated). reading: the pages name
+    no optimizer; the fused update is plain SGD, with G the bf16 gradient of W, lr an
+    fp32 scalar, and the exact value W - lr * G rounded once to fp32 (nearest, ties to
+    even).
+
+    lr * G is exact in fp64 (24-bit times 8-bit significands). W - lr * G is formed as
+    an fp64 sum s plus its exact error e (Knuth's two-sum), so s + e is the exact value;
+    s rounded to fp32 is the answer unless s lies exactly halfway between two fp32
+    values, where the sign of e decides (e = 0: ties to even).
+    """
+    w64 = np.asarray(w, dtype=np.float32).astype(np.float64)
+    p = -(np.float64(np.float32(lr)) * bf16_to_f32(g_bits).astype(np.float64))   # exact
+    s = w64 + p
+    bv = s - w64
+    e = (w64 - (s - bv)) + (p - bv)                    # s + e == w - lr * g exactly
+    r = s.astype(np.float32)                            # nearest fp32, ties to even
+    r64 = r.astype(np.float64)
+    up = np.nextafter(r, np.float32(np.inf)).astype(np.float64)
+    dn = np.nextafter(r, np.float32(-np.inf)).astype(np.float64)
+    to_up = (s == (r64 + up) / 2) & (e > 0)             # s is the upper midpoint, true value above it
+    to_dn = (s == (r64 + dn) / 2) & (e < 0)             # s is the lower midpoint, true value below it
+    out = r.copy()
+    out[to_up] = up[to_up].astype(np.float32)
+    out[to_dn] = dn[to_dn].astype(np.float32)
+    return out
+
+
+def sgd_quant_mask(w: np.ndarray, g_bits: np.ndarray, lr: float, n_keep: int, m_group: int) -> dict:
+    """The optimizer step fused with steps a1 + a2: the updated W, then exactly
+    ``quant_mask`` of it (Sparse-BitNet article section 三: mask and codes follow
+    the latent weights every step)."""
+    w_new = sgd_update(w, g_bits, lr)
+    out = quant_mask(w_new, n_keep, m_group)
+    out["w"] = w_new
+    return out
+
+
 # --------------------------------------------------------------------------- step a3
 
 def act_quant(x_bits: np.ndarray) -> tuple[np.ndarray, np.ndarray]:

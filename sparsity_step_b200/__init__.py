@@ -21,5 +21,6 @@ from .bitlinear import (  # noqa: F401
     bitlinear_quant_mask_noalloc,
     bitlinear_quant_mask_status,
     bitlinear_quant_mask_workspace_size,
+    bitlinear_sgd_quant_mask,
     sp_meta_shape,
 )

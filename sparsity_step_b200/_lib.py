@@ -26,6 +26,7 @@ _P = _c.c_void_p
 _I64 = _c.c_int64
 _INT = _c.c_int
 _SZ = _c.c_size_t
+_F32 = _c.c_float
 
 class BlFwdProblem(ctypes.Structure):
     """bl_fwd_problem of include/bitlinear.h."""
@@ -38,6 +39,7 @@ class BlFwdProblem(ctypes.Structure):
 SIGNATURES = {
     "bitlinear_quant_mask_workspace_size": (_SZ, [_I64, _I64]),
     "bitlinear_quant_mask": (_INT, [_P, _I64, _I64, _INT, _INT, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "bitlinear_sgd_quant_mask": (_INT, [_P, _P, _F32, _I64, _I64, _INT, _INT, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bitlinear_quant_mask_status": (_INT, [_P, _P]),
     "bitlinear_quant_mask_noalloc": (_INT, [_P, _I64, _I64, _INT, _INT, _P, _P, _P, _P, _P]),
     "bitlinear_act_quant": (_INT, [_P, _I64, _I64, _P, _P, _P]),

@@ -116,6 +116,44 @@ def bitlinear_quant_mask(w: torch.Tensor, n_keep: int, m_group: int, *, want_mas
     return o
 
 
+def bitlinear_sgd_quant_mask(w: torch.Tensor, grad_w: torch.Tensor, lr: float, n_keep: int, m_group: int, *,
+                             want_mask: bool = True, want_w_i8: bool = True, want_sp: bool = False,
+                             out: dict | None = None, workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """One SGD step on the latent weights fused with the mask/code recompute:
+    w <- fp32(w - lr * grad_w) in place (grad_w bf16 [n_out, k_in]), then the outputs of
+    ``bitlinear_quant_mask`` for the updated w."""
+    n_out, k_in = w.shape
+    _need(w, torch.float32, None, "w")
+    _need(grad_w, torch.bfloat16, (n_out, k_in), "grad_w", w.device)
+    dev = w.device
+    o = dict(out or {})
+    if "codes" not in o:
+        o["codes"] = torch.empty((n_out, k_in // 4), dtype=torch.uint8, device=dev)
+    if "w_scale" not in o:
+        o["w_scale"] = torch.empty((4,), dtype=torch.float32, device=dev)[:1]
+    if want_mask and "mask" not in o:
+        o["mask"] = torch.empty((n_out, k_in // m_group), dtype=torch.uint8, device=dev)
+    if want_w_i8 and "w_i8" not in o:
+        o["w_i8"] = torch.empty((n_out, k_in), dtype=torch.int8, device=dev)
+    if want_sp and "sp_values" not in o:
+        o["sp_values"] = torch.empty((n_out, k_in // 2), dtype=torch.int8, device=dev)
+        o["sp_meta"] = torch.empty(sp_meta_shape(n_out, k_in), dtype=torch.uint8, device=dev)
+    if m_group not in (4, 8) or k_in % m_group:
+        raise ValueError(f"m_group must be 4 or 8 and divide k_in (got {m_group})")
+    _check_qm_outputs(o, n_out, k_in, m_group, dev)
+    ws_bytes = bitlinear_quant_mask_workspace_size(n_out, k_in)
+    if workspace is None:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    _need_bytes(workspace, ws_bytes, "workspace", dev)
+    st = lib().bitlinear_sgd_quant_mask(_ptr(w), _ptr(grad_w), float(lr), n_out, k_in, n_keep, m_group,
+                                        _ptr(o.get("mask")), _ptr(o["codes"]), _ptr(o.get("w_i8")),
+                                        _ptr(o.get("sp_values")), _ptr(o.get("sp_meta")), _ptr(o["w_scale"]),
+                                        _ptr(workspace), workspace.numel(), _stream(stream))
+    check(st, "bitlinear_sgd_quant_mask")
+    o["workspace"] = workspace
+    return o
+
+
 def bitlinear_quant_mask_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise and return the range status (0 or BL_ERR_RANGE = -4); no raise."""
     return int(lib().bitlinear_quant_mask_status(_ptr(workspace), _stream(stream)))

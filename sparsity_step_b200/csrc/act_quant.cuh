@@ -12,6 +12,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "cp_async.cuh"
 
 namespace bl {
 
@@ -132,6 +133,74 @@ __global__ void __launch_bounds__(256) act_quant_warp_kernel(const uint4* __rest
     }
     if (lane == 0) absmax_out[row] = a;
   }
+}
+
+// Long rows (k8 > 512) on persistent CTAs: each thread streams its own 16-byte vectors of
+// the CTA's next kD - 1 rows into a shared-memory ring with cp.async while it quantises
+// the current row from the ring, so the loads of later rows stay in flight through the
+// block reduction and the stores of this one. One block barrier per row (the partial
+// maxima alternate between two buffers). Ring: kD rows x VPT vectors x 256 threads x 16 B.
+template <int VPT, int kD>
+__global__ void __launch_bounds__(256) act_quant_ring_kernel(const uint4* __restrict__ x, int64_t t, int k8,
+                                                             int8_t* __restrict__ xq, float* __restrict__ absmax_out) {
+  extern __shared__ __align__(16) uint8_t aq_ring[];
+  __shared__ uint32_t s_red[2][8];
+  const uint32_t base = smem_u32(aq_ring) + threadIdx.x * 16u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto slot = [&](int s, int i) { return base + static_cast<uint32_t>((s * VPT + i) * 256) * 16u; };
+  auto issue = [&](int s, int64_t row) {   // this thread's vectors of `row` into ring slot s
+    if (row < t) {
+      const uint4* xr = x + row * k8;
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const int idx = threadIdx.x + i * 256;
+        if (idx < k8) cp_async16(slot(s, i), xr + idx, true);
+      }
+    }
+    cp_async_commit();
+  };
+  const int64_t step = gridDim.x;
+  int64_t row = blockIdx.x;
+#pragma unroll
+  for (int j = 0; j < kD - 1; ++j) issue(j, row + j * step);
+  for (int it = 0; row < t; ++it, row += step) {
+    const int s = it % kD;
+    issue((it + kD - 1) % kD, row + (kD - 1) * step);
+    cp_async_wait<kD - 1>();   // this thread's copies of `row` have landed
+    uint4 v[VPT];
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = threadIdx.x + i * 256;
+      if (idx < k8) {
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v[i].x), "=r"(v[i].y), "=r"(v[i].z), "=r"(v[i].w)
+                     : "r"(slot(s, i)));
+        m = bf16x2_absmax(v[i].x, m);
+        m = bf16x2_absmax(v[i].y, m);
+        m = bf16x2_absmax(v[i].z, m);
+        m = bf16x2_absmax(v[i].w, m);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) s_red[it & 1][warp] = m;
+    __syncthreads();
+    uint32_t mm = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) mm = max(mm, s_red[it & 1][w]);
+    float a = __uint_as_float(mm << 16);
+    if (a == 0.0f) a = 1e-5f;   // an all-zero row quantises to zeros
+    const float sc = __fdiv_rn(127.0f, a);
+    uint2* out = reinterpret_cast<uint2*>(xq + row * (static_cast<int64_t>(k8) * 8));
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int idx = threadIdx.x + i * 256;
+      if (idx < k8) out[idx] = make_uint2(quant_pack4(v[i].x, v[i].y, sc), quant_pack4(v[i].z, v[i].w, sc));
+    }
+    if (threadIdx.x == 0) absmax_out[row] = a;
+  }
+  cp_async_wait<0>();
 }
 
 // Rows too long to cache in registers: read the row twice (max, then quantise).

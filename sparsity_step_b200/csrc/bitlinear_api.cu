@@ -1,6 +1,7 @@
 // C ABI of the BitLinear path (declared in include/bitlinear.h): argument checks,
 // workspace layout, TMA descriptor encoding and kernel dispatch. No allocation:
 // the caller owns every buffer.
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -331,6 +332,13 @@ struct QmOutputs {
   int64_t k8, meta_pitch;   // metadata bytes per row and its padded row pitch
 };
 
+// The optional latent-weight update fused into pass 1: W <- fp32(W - lr * grad), in place.
+struct QmUpdate {
+  float* w = nullptr;                // the same tensor as the weights read (updated in place)
+  const uint16_t* grad = nullptr;    // bf16 [n_out, k_in]; null: no update
+  float lr = 0.0f;
+};
+
 // Padded extents of the 2:4 metadata: rows and logical K rounded up to 256, so that the
 // sparse product's metadata loads never leave the tensor.
 inline int64_t sp_rows(int64_t n_out) { return (n_out + bl::kSpPad - 1) / bl::kSpPad * bl::kSpPad; }
@@ -376,33 +384,42 @@ void launch_codes(const uint4* w4, int64_t n8, int n_keep, float* gamma, const Q
   }
 }
 
+// Pass 1 for one compile-time N:M, mask choice and update choice.
+template <int M, int NK, bool kMask, bool kUpdate>
+void launch_sum(const uint4* w4, int64_t numel, int n_keep, const QmOutputs& o, const bl::QmScratch& q, float* gamma,
+                const QmUpdate& u, cudaStream_t st) {
+  static int occ = 0;   // per instantiation
+  auto k = bl::qm_sum_mask_kernel<M, NK, kMask, kUpdate>;
+  const int grid = qm_blocks_launch(numel, device_sm_count() * resident_blocks(k, &occ));
+  k<<<grid, bl::kQmThreads, 0, st>>>(w4, numel / 8, numel, n_keep, q, gamma, kMask ? o.mask : nullptr,
+                                    reinterpret_cast<uint4*>(u.w), reinterpret_cast<const uint4*>(u.grad), u.lr);
+}
+
 // Both passes for one compile-time N:M. With a mask output, pass 1 ranks the groups and
 // stores the keep bits there, and pass 2 reads them back; without one, pass 2 ranks.
+// With an update (u.grad set), pass 1 first applies it to W in place.
 // Both grids are one wave of resident blocks (grid-stride loops): a partial second wave
 // would leave most SMs idle at the end of each pass.
 template <int M, int NK>
 void launch_quant_mask(const float* w, int64_t numel, int n_keep, const QmOutputs& o, const bl::QmScratch& q,
-                       float* gamma, cudaStream_t st) {
+                       float* gamma, const QmUpdate& u, cudaStream_t st) {
   const uint4* w4 = reinterpret_cast<const uint4*>(w);
   const int64_t n8 = numel / 8;
-  const int sms = device_sm_count();
-  static int occ1 = 0;   // per instantiation
+  const bool upd = u.grad != nullptr;
   if (o.mask != nullptr) {
-    auto k1 = bl::qm_sum_mask_kernel<M, NK, true>;
-    k1<<<qm_blocks_launch(numel, sms * resident_blocks(k1, &occ1)), bl::kQmThreads, 0, st>>>(w4, n8, numel, n_keep, q,
-                                                                                               gamma, o.mask);
+    if (upd) launch_sum<M, NK, true, true>(w4, numel, n_keep, o, q, gamma, u, st);
+    else launch_sum<M, NK, true, false>(w4, numel, n_keep, o, q, gamma, u, st);
     launch_codes<M, NK, true>(w4, n8, n_keep, gamma, o, st);
   } else {
-    auto k1 = bl::qm_sum_mask_kernel<8, 8, false>;
-    k1<<<qm_blocks_launch(numel, sms * resident_blocks(k1, &occ1)), bl::kQmThreads, 0, st>>>(w4, n8, numel, n_keep, q,
-                                                                                               gamma, nullptr);
+    if (upd) launch_sum<8, 8, false, true>(w4, numel, n_keep, o, q, gamma, u, st);
+    else launch_sum<8, 8, false, false>(w4, numel, n_keep, o, q, gamma, u, st);
     launch_codes<M, NK, false>(w4, n8, n_keep, gamma, o, st);
   }
 }
 
 // Both passes of steps a1 + a2 on `scratch` (its first 16 bytes are cleared here).
 bl_status enqueue_quant_mask(const float* w, int64_t n_out, int64_t k_in, int n_keep, int m_group, const QmOutputs& o,
-                             float* gamma, void* scratch, cudaStream_t st) {
+                             float* gamma, void* scratch, cudaStream_t st, const QmUpdate& u = QmUpdate{}) {
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   cudaError_t e = cudaMemsetAsync(ws, 0, 16, st);   // range flag, status, blocks-done ticket
   if (e != cudaSuccess) return cuda_fail(e, "scratch reset");
@@ -412,21 +429,21 @@ bl_status enqueue_quant_mask(const float* w, int64_t n_out, int64_t k_in, int n_
                         reinterpret_cast<unsigned long long*>(ws + bl::kQmWsHeader)};
   if (m_group == 8) {
     switch (n_keep) {
-      case 8: launch_quant_mask<8, 8>(w, numel, n_keep, o, q, gamma, st); break;
-      case 7: launch_quant_mask<8, 7>(w, numel, n_keep, o, q, gamma, st); break;
-      case 6: launch_quant_mask<8, 6>(w, numel, n_keep, o, q, gamma, st); break;
-      case 5: launch_quant_mask<8, 5>(w, numel, n_keep, o, q, gamma, st); break;
-      case 4: launch_quant_mask<8, 4>(w, numel, n_keep, o, q, gamma, st); break;
-      case 3: launch_quant_mask<8, 3>(w, numel, n_keep, o, q, gamma, st); break;
-      case 2: launch_quant_mask<8, 2>(w, numel, n_keep, o, q, gamma, st); break;
-      default: launch_quant_mask<8, 1>(w, numel, n_keep, o, q, gamma, st); break;
+      case 8: launch_quant_mask<8, 8>(w, numel, n_keep, o, q, gamma, u, st); break;
+      case 7: launch_quant_mask<8, 7>(w, numel, n_keep, o, q, gamma, u, st); break;
+      case 6: launch_quant_mask<8, 6>(w, numel, n_keep, o, q, gamma, u, st); break;
+      case 5: launch_quant_mask<8, 5>(w, numel, n_keep, o, q, gamma, u, st); break;
+      case 4: launch_quant_mask<8, 4>(w, numel, n_keep, o, q, gamma, u, st); break;
+      case 3: launch_quant_mask<8, 3>(w, numel, n_keep, o, q, gamma, u, st); break;
+      case 2: launch_quant_mask<8, 2>(w, numel, n_keep, o, q, gamma, u, st); break;
+      default: launch_quant_mask<8, 1>(w, numel, n_keep, o, q, gamma, u, st); break;
     }
   } else {
     switch (n_keep) {
-      case 4: launch_quant_mask<4, 4>(w, numel, n_keep, o, q, gamma, st); break;
-      case 3: launch_quant_mask<4, 3>(w, numel, n_keep, o, q, gamma, st); break;
-      case 2: launch_quant_mask<4, 2>(w, numel, n_keep, o, q, gamma, st); break;
-      default: launch_quant_mask<4, 1>(w, numel, n_keep, o, q, gamma, st); break;
+      case 4: launch_quant_mask<4, 4>(w, numel, n_keep, o, q, gamma, u, st); break;
+      case 3: launch_quant_mask<4, 3>(w, numel, n_keep, o, q, gamma, u, st); break;
+      case 2: launch_quant_mask<4, 2>(w, numel, n_keep, o, q, gamma, u, st); break;
+      default: launch_quant_mask<4, 1>(w, numel, n_keep, o, q, gamma, u, st); break;
     }
   }
   e = cudaGetLastError();
@@ -474,6 +491,31 @@ int qm_blocks_launch(int64_t numel, int resident) {
   return b < bound ? b : bound;
 }
 
+// Rows of 513..2048 vectors: the persistent ring kernel, a three-row ring per CTA and as
+// many CTAs as fit on an SM (shared memory decides), one wave.
+template <int VPT>
+bl_status launch_act_quant_ring(const uint4* xv, int64_t t, int k8, int8_t* xq_out, float* absmax_out,
+                                cudaStream_t st) {
+  constexpr int kD = 3;
+  constexpr int smem = kD * VPT * 256 * 16;
+  static int occ = 0;   // per instantiation
+  if (occ <= 0) {
+    cudaError_t e = cudaFuncSetAttribute(bl::act_quant_ring_kernel<VPT, kD>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(act_quant ring)");
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bl::act_quant_ring_kernel<VPT, kD>, 256, smem) !=
+            cudaSuccess ||
+        n <= 0)
+      n = 1;
+    occ = n;
+  }
+  int64_t grid = int64_t(device_sm_count()) * occ;
+  if (grid > t) grid = t;
+  bl::act_quant_ring_kernel<VPT, kD><<<static_cast<unsigned>(grid), 256, smem, st>>>(xv, t, k8, xq_out, absmax_out);
+  return BL_OK;
+}
+
 // Launch of the act_quant kernels (arguments already checked).
 bl_status enqueue_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t* xq_out, float* absmax_out,
                             cudaStream_t st) {
@@ -491,12 +533,14 @@ bl_status enqueue_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t* 
     else bl::act_quant_warp_kernel<16><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
   } else {   // one CTA per row
     const int vpt = (k8 + 255) / 256;
-    if (vpt <= 4) bl::act_quant_kernel<4, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-    else if (vpt <= 6) bl::act_quant_kernel<6, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-    else if (vpt <= 8) bl::act_quant_kernel<8, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
+    bl_status s = BL_OK;
+    if (vpt <= 4) s = launch_act_quant_ring<4>(xv, t, k8, xq_out, absmax_out, st);
+    else if (vpt <= 6) s = launch_act_quant_ring<6>(xv, t, k8, xq_out, absmax_out, st);
+    else if (vpt <= 8) s = launch_act_quant_ring<8>(xv, t, k8, xq_out, absmax_out, st);
     else if (vpt <= 12) bl::act_quant_kernel<12, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
     else if (vpt <= 16) bl::act_quant_kernel<16, 1><<<g1, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
     else bl::act_quant_long_kernel<<<g1, 256, 0, st>>>(xv, k8, xq_out, absmax_out);
+    if (s != BL_OK) return s;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
@@ -653,6 +697,39 @@ bl_status bitlinear_quant_mask(const float* w_latent, int64_t n_out, int64_t k_i
     return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
   const QmOutputs o{mask_out, codes_out, w_i8_out, sp_values_out, sp_meta_out, k_in / 8, sp_meta_pitch(k_in)};
   return enqueue_quant_mask(w_latent, n_out, k_in, n_keep, m_group, o, w_scale_out, workspace, as_stream(stream));
+}
+
+bl_status bitlinear_sgd_quant_mask(float* w_latent, const uint16_t* grad_w, float lr, int64_t n_out, int64_t k_in,
+                                   int n_keep, int m_group, uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out,
+                                   int8_t* sp_values_out, uint8_t* sp_meta_out, float* w_scale_out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  if (!grad_w) return fail(BL_ERR_INVALID_ARG, "grad_w is required");
+  if (!std::isfinite(lr)) return fail(BL_ERR_INVALID_ARG, "lr must be finite");
+  if (!aligned16(grad_w)) return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  if (!w_latent || !codes_out || !w_scale_out) return fail(BL_ERR_INVALID_ARG, "w_latent, codes_out, w_scale_out are required");
+  if (bl_status s = check_shape(0, k_in, n_out)) return s;
+  if (!(m_group == 4 || m_group == 8) || n_keep < 1 || n_keep > m_group)
+    return fail(BL_ERR_INVALID_ARG, "N:M = %d:%d: need M in {4, 8} and 1 <= N <= M", n_keep, m_group);
+  if ((sp_values_out == nullptr) != (sp_meta_out == nullptr))
+    return fail(BL_ERR_INVALID_ARG, "give both sp_values_out and sp_meta_out, or neither");
+  if (sp_values_out && n_keep > 2)
+    return fail(BL_ERR_INVALID_ARG, "N:M = %d:%d is not 2:4-valid (at most 2 kept per aligned 4): no 2:4 storage",
+                n_keep, m_group);
+  if (!workspace) return fail(BL_ERR_WORKSPACE, "workspace is required");
+  if (workspace_bytes < bitlinear_quant_mask_workspace_size(n_out, k_in))
+    return fail(BL_ERR_WORKSPACE, "workspace too small: %zu < %zu", workspace_bytes,
+                bitlinear_quant_mask_workspace_size(n_out, k_in));
+  if (!aligned16(w_latent) || !aligned16(codes_out) || !aligned16(w_scale_out) || !aligned16(workspace) ||
+      (mask_out && !aligned16(mask_out)) || (w_i8_out && !aligned16(w_i8_out)) ||
+      (sp_values_out && !aligned16(sp_values_out)) || (sp_meta_out && !aligned16(sp_meta_out)))
+    return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  const QmOutputs o{mask_out, codes_out, w_i8_out, sp_values_out, sp_meta_out, k_in / 8, sp_meta_pitch(k_in)};
+  QmUpdate u;
+  u.w = w_latent;
+  u.grad = grad_w;
+  u.lr = lr;
+  return enqueue_quant_mask(w_latent, n_out, k_in, n_keep, m_group, o, w_scale_out, workspace, as_stream(stream), u);
 }
 
 bl_status bitlinear_quant_mask_status(const void* workspace, void* stream) {

@@ -12,6 +12,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "cp_async.cuh"
 
 namespace bl {
 
@@ -230,16 +231,6 @@ __device__ __forceinline__ DecTask dec_task(const FwdGroup& G, int task, int tok
   d.nch = (P.k_in + 255) >> 8;
   return d;
 }
-
-// 16-byte async copy global -> shared; `valid` false writes zeros (src not read). No
-// compiler memory barrier: ordering comes from the commit and wait that follow.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
-               "r"(valid ? 16 : 0));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int NG>   // token groups of 8 per task
 __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(const __grid_constant__ FwdGroup G) {

@@ -408,23 +408,62 @@ __host__ __device__ __forceinline__ QmCodes8 qm_codes8(const uint32_t (&b)[8], u
   return r;
 }
 
+// Optimizer step of the latent weights fused into pass 1 (kUpdate): W <- fp32(W - lr * G)
+// with G the bf16 gradient, one fused multiply-add (a single rounding) per weight; the
+// updated weights are stored back and summed and ranked in the same pass, so the mask
+// recompute costs no extra read of W. Loads of W then use the coherent path (the kernel
+// writes W). `step` holds the 8 weights of one thread step and their 8 gradients.
+struct QmStepIn {
+  QmPair w;
+  uint4 g;
+};
+template <bool kUpdate>
+__device__ __forceinline__ QmStepIn qm_load_step(const uint4* w4, const uint4* g4, int64_t g, bool ok) {
+  QmStepIn v{{make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)}, make_uint4(0, 0, 0, 0)};
+  if (!kUpdate) {
+    v.w = qm_load(w4, g, ok);
+  } else if (ok) {
+    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.w.lo.x), "=r"(v.w.lo.y), "=r"(v.w.lo.z), "=r"(v.w.lo.w)
+                 : "l"(w4 + 2 * g));
+    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.w.hi.x), "=r"(v.w.hi.y), "=r"(v.w.hi.z), "=r"(v.w.hi.w)
+                 : "l"(w4 + 2 * g + 1));
+    v.g = ld_nc_u4(g4 + g);
+  }
+  return v;
+}
+
 // Pass 1: exact integer sum of floor(|w| * 2^32) and, with kMask, the keep bits of
 // every group stored to `mask`. Each block stores its partial sum; the last block to
 // finish (atomic ticket) adds all partials, rounds the mean once to fp32, writes
 // gamma = mean + 1e-5 (NaN and status BL_ERR_RANGE on a range error) and clears the
 // ticket and the flag for the next call. Two thread steps are in flight per thread
-// (register double buffer; loads past the end give zeros, which add nothing).
-template <int M, int NK, bool kMask>
-__global__ void __launch_bounds__(kQmThreads) qm_sum_mask_kernel(const uint4* __restrict__ w4, int64_t n8,
+// (register double buffer; loads past the end give zeros, which add nothing). With
+// kUpdate, `w4` is updated in place first (see above).
+template <int M, int NK, bool kMask, bool kUpdate>
+__global__ void __launch_bounds__(kQmThreads) qm_sum_mask_kernel(const uint4* w4, int64_t n8,
                                                                   int64_t numel, int n_keep, QmScratch ws,
                                                                   float* __restrict__ gamma_out,
-                                                                  uint8_t* __restrict__ mask) {
+                                                                  uint8_t* __restrict__ mask, uint4* w4_out,
+                                                                  const uint4* __restrict__ g4, float lr) {
   static_assert(M == 4 || M == 8, "groups of 4 or 8");
   uint64_t acc = 0;
   uint32_t bad = 0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  auto step = [&](const QmPair& v, int64_t g) {
-    const uint32_t b[8] = {v.lo.x, v.lo.y, v.lo.z, v.lo.w, v.hi.x, v.hi.y, v.hi.z, v.hi.w};
+  const float neg_lr = -lr;
+  auto step = [&](const QmStepIn& v, int64_t g) {
+    uint32_t b[8] = {v.w.lo.x, v.w.lo.y, v.w.lo.z, v.w.lo.w, v.w.hi.x, v.w.hi.y, v.w.hi.z, v.w.hi.w};
+    if (kUpdate) {
+      const uint32_t gw[4] = {v.g.x, v.g.y, v.g.z, v.g.w};   // bf16 pairs: element 2i low, 2i+1 high
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float gj = __uint_as_float((j & 1) ? (gw[j >> 1] & 0xffff0000u) : (gw[j >> 1] << 16));
+        b[j] = __float_as_uint(__fmaf_rn(neg_lr, gj, __uint_as_float(b[j])));
+      }
+      w4_out[2 * g] = make_uint4(b[0], b[1], b[2], b[3]);
+      w4_out[2 * g + 1] = make_uint4(b[4], b[5], b[6], b[7]);
+    }
     qm_accumulate8(b, acc, bad);
     if (kMask) {
       const uint32_t keep = qm_keep8<M, NK>(b, n_keep);
@@ -433,12 +472,12 @@ __global__ void __launch_bounds__(kQmThreads) qm_sum_mask_kernel(const uint4* __
     }
   };
   int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  QmPair va = qm_load(w4, g, g < n8), vb;
+  QmStepIn va = qm_load_step<kUpdate>(w4, g4, g, g < n8), vb;
   for (; g < n8; g += 2 * stride) {
-    vb = qm_load(w4, g + stride, g + stride < n8);
+    vb = qm_load_step<kUpdate>(w4, g4, g + stride, g + stride < n8);
     step(va, g);
     if (g + stride >= n8) break;
-    va = qm_load(w4, g + 2 * stride, g + 2 * stride < n8);
+    va = qm_load_step<kUpdate>(w4, g4, g + 2 * stride, g + 2 * stride < n8);
     step(vb, g + stride);
   }
   if (bad & 0x80000000u) atomicOr(ws.range_flag, 1u);   // |w| >= 2^16, inf or NaN

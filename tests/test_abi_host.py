@@ -58,6 +58,24 @@ def test_quant_mask_validation(L):
     assert "aligned" in _err(L)
 
 
+def test_sgd_quant_mask_validation(L):
+    ws = L.bitlinear_quant_mask_workspace_size(896, 896)
+    call = L.bitlinear_sgd_quant_mask
+    # the gradient and a finite learning rate are required
+    assert call(GOOD, None, 1e-3, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -1
+    for lr in (float("nan"), float("inf")):
+        assert call(GOOD, GOOD, lr, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -1
+        assert "lr" in _err(L)
+    assert call(GOOD, BAD, 1e-3, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -3
+    # then the checks of bitlinear_quant_mask
+    assert call(None, GOOD, 1e-3, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -1
+    assert call(GOOD, GOOD, 1e-3, 896, 896, 9, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -1
+    assert call(GOOD, GOOD, 1e-3, 896, 900, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -2
+    assert call(GOOD, GOOD, 1e-3, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws - 1, None) == -7
+    assert call(GOOD, GOOD, 1e-3, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, ws, None) == -1
+    assert call(BAD, GOOD, 1e-3, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -3
+
+
 def test_quant_mask_noalloc_validation(L):
     assert L.bitlinear_quant_mask_noalloc(None, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, None) == -1
     assert L.bitlinear_quant_mask_noalloc(GOOD, 896, 896, 9, 8, GOOD, GOOD, GOOD, GOOD, None) == -1

@@ -584,3 +584,59 @@ def test_compress_2_4_rejects_denser_masks(n, m):
     qm = O.quant_mask(w, n, m)
     with pytest.raises(ValueError):
         O.compress_2_4(qm["mcode"], qm["keep"])
+
+
+# ----------------------------------------------------------------------- optimizer step
+
+def _rn_f32_exact(v: Fraction) -> float:
+    """Nearest fp32 to the rational v (ties to the even significand), by comparing v
+    with the candidates around fl64(v) in exact arithmetic (independent of the
+    oracle's two-sum method)."""
+    c = np.float32(float(v))
+    cands = {float(c), float(np.nextafter(c, np.float32(np.inf))), float(np.nextafter(c, np.float32(-np.inf)))}
+    best = None
+    for x in sorted(cands):
+        d = abs(Fraction(x) - v)
+        even = (int(np.array(x, dtype=np.float32).view(np.uint32)) & 1) == 0
+        key = (d, not even)
+        if best is None or key < best[0]:
+            best = (key, x)
+    return best[1]
+
+
+def test_hand_sgd_update_ties_and_sticky_error():
+    """Golden rows sgd_*: plain SGD rounds W - lr*G once; cases 5 and 6 are a quarter
+    fp64 ulp above an fp32 halfway point, where rounding an fp64 sum would tie to even."""
+    w = np.array([float(t) for t in G["sgd_w"]], dtype=np.float32)
+    g = synth.f32_to_bf16_bits(np.array([float(t) for t in G["sgd_g"]], dtype=np.float32))
+    want = np.array([float(t) for t in G["sgd_w_new"]], dtype=np.float32)
+    for i, lr in enumerate(float(t) for t in G["sgd_lr"]):
+        got = O.sgd_update(w[i:i + 1], g[i:i + 1], lr)
+        assert got[0] == want[i], (i, float(got[0]), float(want[i]))
+
+
+def test_sgd_update_brute_force_exact_rationals():
+    """Random W (magnitudes 2^-20 .. 2^10), bf16 G and fp32 lr, including exponent gaps
+    wider than fp64 holds: the oracle equals the exactly rounded rational W - lr*G."""
+    rng = np.random.default_rng(7)
+    n = 4000
+    w = (rng.standard_normal(n) * np.exp2(rng.integers(-20, 10, n))).astype(np.float32)
+    gf = (rng.standard_normal(n) * np.exp2(rng.integers(-12, 6, n))).astype(np.float32)
+    g = synth.f32_to_bf16_bits(gf)
+    lrs = (np.exp2(rng.integers(-40, 0, n)) * rng.uniform(0.5, 1.0, n)).astype(np.float32)
+    gv = O.bf16_to_f32(g)
+    for i in range(n):
+        got = O.sgd_update(w[i:i + 1], g[i:i + 1], float(lrs[i]))[0]
+        exact = Fraction(float(w[i])) - Fraction(float(lrs[i])) * Fraction(float(gv[i]))
+        assert float(got) == _rn_f32_exact(exact), (float(w[i]), float(lrs[i]), float(gv[i]))
+
+
+def test_sgd_quant_mask_zero_step_is_quant_mask():
+    """lr = 0 leaves W unchanged, so the fused step reduces to the plain mask/code step."""
+    w = synth.latent_weight(3, 16, 64)
+    g = synth.activation_bf16(4, 16, 64)
+    a = O.sgd_quant_mask(w, g, 0.0, 6, 8)
+    b = O.quant_mask(w, 6, 8)
+    assert np.array_equal(a["w"], w)
+    assert a["gamma"] == b["gamma"] and np.array_equal(a["codes_packed"], b["codes_packed"])
+    assert np.array_equal(a["mask"], b["mask"])

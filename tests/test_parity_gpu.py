@@ -398,6 +398,67 @@ def test_range_error_reported():
     check_quant_mask(out, O.quant_mask(w, 6, 8), "after range error")
 
 
+# ------------------------------------------------------------------ optimizer step fused with the mask recompute
+
+
+def gpu_sgd_quant_mask(w_np, g_bits, lr, n, m):
+    wd = f32_to_dev(w_np)
+    out = B.bitlinear_sgd_quant_mask(wd, bits_to_dev_bf16(g_bits), lr, n, m, want_sp=n <= 2)
+    torch.cuda.synchronize()
+    assert B.bitlinear_quant_mask_status(out["workspace"]) == 0
+    return wd.cpu().numpy(), out
+
+
+@pytest.mark.parametrize("nm", [(6, 8), (2, 4), (8, 8)], ids=lambda v: f"{v[0]}of{v[1]}")
+@pytest.mark.parametrize("n_out,k_in", [(272, 896), (16, 64)])
+def test_sgd_quant_mask_small(n_out, k_in, nm):
+    """W <- fp32(W - lr*G) in place (bit-exact), then gamma, mask, codes and int8 codes
+    of the updated W (bit-exact)."""
+    n, m = nm
+    w = synth.latent_weight(120, n_out, k_in)
+    g = synth.activation_bf16(121, n_out, k_in)
+    lr = 3e-3
+    ref = O.sgd_quant_mask(w, g, lr, n, m)
+    w_new, out = gpu_sgd_quant_mask(w, g, lr, n, m)
+    assert_exact(w_new.view(np.uint32), ref["w"].view(np.uint32), "updated W")
+    check_quant_mask(out, ref, f"sgd {n}:{m}")
+
+
+def test_sgd_update_rounding_cases():
+    """The hand-worked SGD cases (halfway points; a quarter fp64 ulp above one) on the
+    device: one fused multiply-add rounds like the exact value."""
+    cases = [(1.0, 2.0 ** -24, -1.0, 1.0), (1.0, 2.0 ** -24, -1.0078125, 1.0 + 2.0 ** -23),
+             (1.0 + 2.0 ** -23, 2.0 ** -24, 1.0, 1.0), (1.0, 16519105 * 2.0 ** -48, -1.015625, 1.0 + 2.0 ** -23),
+             (1.0 + 2.0 ** -23, 7110873 * 2.0 ** -47, 1.1796875, 1.0 + 2.0 ** -23)]
+    for w0, lr, g0, want in cases:
+        w = np.full((16, 64), w0, np.float32)
+        g = synth.f32_to_bf16_bits(np.full((16, 64), g0, np.float32))
+        w_new, out = gpu_sgd_quant_mask(w, g, lr, 6, 8)
+        assert np.all(w_new == np.float32(want)), (w0, lr, g0)
+        check_quant_mask(out, O.sgd_quant_mask(w, g, lr, 6, 8), f"sgd case {w0} {lr} {g0}")
+
+
+def test_sgd_quant_mask_training_shape():
+    """The 3B MLP gate projection (11008 x 2048), one step: the whole updated W and gamma
+    bit-exact, mask and codes on sampled rows."""
+    n_out, k_in = 11008, 2048
+    w = synth.latent_weight(122, n_out, k_in)
+    g = synth.activation_bf16(123, n_out, k_in, std=1e-2, outliers=False)
+    lr = 0.05
+    w_ref = O.sgd_update(w, g, lr)
+    w_new, out = gpu_sgd_quant_mask(w, g, lr, 6, 8)
+    assert_exact(w_new.view(np.uint32), w_ref.view(np.uint32), "updated W")
+    gamma, _, _ = O.absmean_gamma(w_ref)
+    assert_exact(out["w_scale"].cpu().numpy()[:1].view(np.uint32), np.array([gamma], np.float32).view(np.uint32), "gamma")
+    rows = sample_rows(n_out, 5)
+    code = O.ternary_codes(w_ref[rows], gamma)
+    keep = O.nm_keep(w_ref[rows], 6, 8)
+    mcode = (code * keep).astype(np.int8)
+    assert_exact(out["mask"].cpu().numpy()[rows], O.mask_bytes(keep, 8), "mask")
+    assert_exact(out["codes"].cpu().numpy()[rows], O.pack_codes(mcode), "codes")
+    assert_exact(out["w_i8"].cpu().numpy()[rows], mcode, "w_i8")
+
+
 def test_no_device_timeouts():
     st, bits = B.bitlinear_device_status()
     assert st == 0 and bits == 0
