@@ -437,16 +437,17 @@ def run_ours(args) -> None:
         probe = {"error": str(exc)}
 
     # ---------------- roofline of the dominant kernel
-    # Peak: the measured burst bf16 rate when the timed region is short or the SM clock
-    # stayed near its maximum (the kernel ran at the clock the burst figure was taken
-    # at); the sustained (power-capped) rate only for a long region at lowered clocks.
+    # Peak: the measured burst bf16 rate when the SM clock stayed near its maximum (the
+    # kernels ran at the clock the burst figure was taken at); the sustained
+    # (power-capped) rate when the power cap lowered the clock during the timed region.
+    # Without a clock record, a region under a second counts as a burst.
     peaks = load_peaks()
     fwd_ops, bwd_flops = algorithmic_counts()
     dominant = max(per_kernel_ms, key=per_kernel_ms.get)
     gemm_flops_per_launch = 2 * TOKENS * 2048 * 11008          # every product here has this size
     smhz, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
     at_max_clock = bool(smhz and smax and smhz >= 0.95 * smax)
-    use_burst = ms_total < 1000.0 or at_max_clock
+    use_burst = at_max_clock if (smhz and smax) else ms_total < 1000.0
     bf16_peak = peaks["bf16_tflops"] if use_burst else peaks["bf16_tflops_sustained"]
     why = ("timed region %.0f ms, median SM clock %s of max %s MHz" % (ms_total, smhz, smax))
     roof = None
@@ -464,9 +465,9 @@ def run_ours(args) -> None:
             roof["frac_vs_tcgen05_probe"] = round(achieved / probe["bf16_tflops"], 4)
     else:
         roof = {"kernel": dominant, "bound": "unknown"}
-    # INT8: no measured peak in the driver's file; derived as 2 x the measured burst bf16
-    # rate (the nominal int8 / bf16 ratio of B200), with this run's tcgen05 probe beside it
-    int8_peak = 2 * peaks["bf16_tflops"]
+    # INT8: no measured peak in the driver's file; derived as 2 x the bf16 rate chosen above (the
+    # nominal int8 / bf16 ratio of B200), with this run's tcgen05 probe beside it
+    int8_peak = 2 * bf16_peak
     fwd_tops = fwd_ops / (per_kernel_ms["fwd_i8_gemm"] * 1e-3) / 1e12
 
     tok_s = job_tokens_per_s(ms_step, world)
@@ -490,7 +491,8 @@ def run_ours(args) -> None:
                  "fwd_int8_useful_6of8": round(fwd_tops * N_KEEP / M_GROUP, 1),
                  "bwd_bf16": round(bwd_flops / ((per_kernel_ms["bwd_grad_x"] + per_kernel_ms["bwd_grad_w"]) * 1e-3) / 1e12, 1),
                  "int8_peak_derived": round(int8_peak, 1),
-                 "int8_peak_kind": "2 x measured burst bf16 (nominal int8/bf16 ratio), not measured",
+                 "int8_peak_kind": f"2 x measured {'burst' if use_burst else 'sustained'} bf16 (nominal int8/bf16 "
+                                   "ratio), not measured",
                  "fwd_frac_of_int8_peak_derived": round(fwd_tops / int8_peak, 4),
                  "fwd_frac_of_int8_probe": (round(fwd_tops / probe["int8_tops"], 4) if "int8_tops" in probe else None),
                  "tensor_pipe_probe": probe},

@@ -16,22 +16,24 @@
 
 namespace bl {
 
-__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t w, uint32_t m) {
-  const uint32_t lo = w & 0x7fffu, hi = (w >> 16) & 0x7fffu;
-  return max(m, max(lo, hi));
+// Running max of |bf16| bit patterns, both halves at once (16-bit SIMD max; the high
+// half is folded in by bf16_absmax_final).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t w, uint32_t m) { return __vmaxu2(m, w & 0x7fff7fffu); }
+__device__ __forceinline__ uint32_t bf16_absmax_final(uint32_t m) { return max(m & 0xffffu, m >> 16); }
+
+// q = clamp(rint(x * s), -128, 127): one fp32 multiply, then one conversion that rounds
+// to nearest even and saturates to int8 (the low byte of the result).
+__device__ __forceinline__ uint32_t quant_one(float xf, float s) {
+  uint32_t q;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(__fmul_rn(xf, s)));
+  return q;
 }
 
-__device__ __forceinline__ int quant_one(uint32_t bf16_bits, float s) {
-  const float xf = __uint_as_float(bf16_bits << 16);
-  const int q = __float2int_rn(__fmul_rn(xf, s));   // round half to even
-  return min(127, max(-128, q));
-}
-
+// Four bf16 (two words) -> four int8 in one word (element 0 in byte 0).
 __device__ __forceinline__ uint32_t quant_pack4(uint32_t w0, uint32_t w1, float s) {
-  const int q0 = quant_one(w0 & 0xffffu, s), q1 = quant_one(w0 >> 16, s);
-  const int q2 = quant_one(w1 & 0xffffu, s), q3 = quant_one(w1 >> 16, s);
-  return (static_cast<uint32_t>(q0) & 0xffu) | ((static_cast<uint32_t>(q1) & 0xffu) << 8) |
-         ((static_cast<uint32_t>(q2) & 0xffu) << 16) | ((static_cast<uint32_t>(q3) & 0xffu) << 24);
+  const uint32_t q0 = quant_one(__uint_as_float(w0 << 16), s), q1 = quant_one(__uint_as_float(w0 & 0xffff0000u), s);
+  const uint32_t q2 = quant_one(__uint_as_float(w1 << 16), s), q3 = quant_one(__uint_as_float(w1 & 0xffff0000u), s);
+  return __byte_perm(__byte_perm(q0, q1, 0x0040u), __byte_perm(q2, q3, 0x0040u), 0x5410u);
 }
 
 __device__ __forceinline__ uint32_t block_max_u32(uint32_t m, uint32_t* s_red) {
@@ -74,6 +76,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const uint4* __restrict_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
+    m[r] = bf16_absmax_final(m[r]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m[r] = max(m[r], __shfl_xor_sync(0xffffffffu, m[r], off));
     if (lane == 0) s_red[r][warp] = m[r];
@@ -98,8 +101,8 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const uint4* __restrict_
 }
 
 // Short rows (k8 <= 32 * VPT): one warp per row, the row held in registers (VPT
-// 16-byte vectors per lane), warp-shuffle max, no block barrier. Persistent warps
-// stride over the rows.
+// 16-byte vectors per lane), warp-shuffle max, no block barrier. Warps stride over the
+// rows; the launch gives every row its own warp.
 template <int VPT>
 __global__ void __launch_bounds__(256) act_quant_warp_kernel(const uint4* __restrict__ x, int64_t t, int k8,
                                                              int8_t* __restrict__ xq, float* __restrict__ absmax_out) {
@@ -120,6 +123,7 @@ __global__ void __launch_bounds__(256) act_quant_warp_kernel(const uint4* __rest
         m = bf16x2_absmax(v[i].w, m);
       }
     }
+    m = bf16_absmax_final(m);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
     float a = __uint_as_float(m << 16);
@@ -182,6 +186,7 @@ __global__ void __launch_bounds__(256) act_quant_ring_kernel(const uint4* __rest
         m = bf16x2_absmax(v[i].w, m);
       }
     }
+    m = bf16_absmax_final(m);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
     if (lane == 0) s_red[it & 1][warp] = m;
@@ -217,7 +222,7 @@ __global__ void __launch_bounds__(256) act_quant_long_kernel(const uint4* __rest
     m = bf16x2_absmax(v.z, m);
     m = bf16x2_absmax(v.w, m);
   }
-  m = block_max_u32(m, s_red);
+  m = block_max_u32(bf16_absmax_final(m), s_red);
   float a = __uint_as_float(m << 16);
   if (a == 0.0f) a = 1e-5f;
   const float s = __fdiv_rn(127.0f, a);
