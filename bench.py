@@ -42,11 +42,14 @@ CFG_INDEX = 4   # the training-step workload's seed block
 # SHA-256 of the kernel's source files at capture time (reported as null once the
 # source has changed).
 TRAFFIC = {
-    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum (1 pass) on the full-size
-    # grad_W launch (16384 x 2048 x 11008, CTA-pair kernel, raster by operand size,
-    # serpentine K): 640,313,856 B read + 41,900,800 B written (the 11008 -> 2048 launch:
-    # 640,384,000 + 42,234,368)
-    "bwd_grad_w": {"sha": "da1ce434dceb301b", "bytes": 682214656},
+    # DRAM bytes per launch from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum`
+    # (1 pass) on the full-size launches of the current GEMM source (see profiles/);
+    # reported only while the kernel source hashes to `sha`.
+    # grouped grad_W (gate, up, down over 16384 tokens): 2,072,903,680 read + 129,520,640 written
+    "bwd_grad_w": {"sha": "dcba4d5a127e6863", "bytes": 2202424320},
+    # grad_X GEMM (16384 x 2048 <- 11008; the code expansion is a separate kernel):
+    # 585,053,696 read + 61,331,712 written
+    "bwd_grad_x": {"sha": "dcba4d5a127e6863", "bytes": 646385408},
 }
 
 
@@ -238,9 +241,10 @@ class Step:
         self.gw = {n: torch.empty((n_out, k_in), dtype=bf, device=dev) for n, k_in, n_out in LINEARS}
         wsb = max(B.bitlinear_bwd_workspace_size(T, k, n, True) for _, k, n in LINEARS)
         self.ws_bwd = torch.empty((wsb,), dtype=torch.uint8, device=dev)
-        # kernels per step: quant_mask 2 (plus a 16-byte memset, not a kernel), act_quant 1,
-        # fwd 1, grad_X 2 (expand + GEMM), grad_W 1
-        self.launches_per_step = 3 * 2 + 2 + 3 + 3 * 2 + 3
+        # kernels per step: quant_mask 2 per weight (plus a 16-byte memset, not a kernel),
+        # act_quant 1 per input width, fwd 1 per linear, grad_X 2 per linear (expand + GEMM),
+        # grad_W 1 for all three linears
+        self.launches_per_step = 3 * 2 + 2 + 3 + 3 * 2 + 1
 
     def run(self, ev=None, io=0):
         """Enqueue one step on the current stream using I/O set ``io``. ``ev`` maps a
@@ -272,12 +276,14 @@ class Step:
             q = self.qm[name]
             timed("fwd_i8_gemm", lambda: B.bitlinear_fwd(xq, a, q["w_scale"], w_i8=q["w_i8"], y=y[name]))
         for name, k_in, _ in LINEARS:
-            x = d["x_down"] if name == "down" else d["x_in"]
             q = self.qm[name]
             dy = d[f"dy_{name}"]
             timed("bwd_grad_x", lambda: B.bitlinear_bwd(dy, None, q["codes"], q["w_scale"], want_grad_w=False,
                                                         grad_x=gx[name], workspace=self.ws_bwd, k_in=k_in))
-            timed("bwd_grad_w", lambda: B.bitlinear_bwd(dy, x, None, None, want_grad_x=False, grad_w=self.gw[name]))
+        # the three weight gradients share the token batch: one launch schedules all their tiles
+        timed("bwd_grad_w", lambda: B.bitlinear_grad_w_grouped(
+            [{"dy": d[f"dy_{name}"], "x": d["x_down"] if name == "down" else d["x_in"], "grad_w": self.gw[name]}
+             for name, _, _ in LINEARS]))
 
     def outputs(self, io=0):
         return [self.io[io]["y"][n] for n, _, _ in LINEARS] + [self.io[io]["gx"][n] for n, _, _ in LINEARS]
@@ -443,28 +449,37 @@ def run_ours(args) -> None:
     # Without a clock record, a region under a second counts as a burst.
     peaks = load_peaks()
     fwd_ops, bwd_flops = algorithmic_counts()
-    dominant = max(per_kernel_ms, key=per_kernel_ms.get)
-    gemm_flops_per_launch = 2 * TOKENS * 2048 * 11008          # every product here has this size
+    gemm_flops = 2 * TOKENS * 2048 * 11008          # every product here has this size
+    # one bwd_grad_w launch computes all three weight gradients; a bwd_grad_x call is one
+    # product (its time includes the 2-bit code expansion that feeds it)
+    flops_per_launch = {"bwd_grad_w": 3 * gemm_flops, "bwd_grad_x": gemm_flops}
     smhz, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
     at_max_clock = bool(smhz and smax and smhz >= 0.95 * smax)
     use_burst = at_max_clock if (smhz and smax) else ms_total < 1000.0
     bf16_peak = peaks["bf16_tflops"] if use_burst else peaks["bf16_tflops_sustained"]
     why = ("timed region %.0f ms, median SM clock %s of max %s MHz" % (ms_total, smhz, smax))
-    roof = None
-    if dominant in ("bwd_grad_w", "bwd_grad_x"):
-        achieved = gemm_flops_per_launch / (per_launch_ms[dominant] * 1e-3) / 1e12
-        tr = TRAFFIC.get(dominant)
-        roof = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_peak,
-                "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
-                "peak_kind": f"bf16 {'burst' if use_burst else 'sustained'} ({peaks['source']}; {why})",
-                "frac_vs_burst": round(achieved / peaks["bf16_tflops"], 4),
-                "frac_vs_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
-                "traffic": tr["bytes"] if tr and tr["sha"] == kernel_source_sha() else None,
-                "algorithmic_per_launch": gemm_flops_per_launch}
+
+    def gemm_roofline(cls):
+        achieved = flops_per_launch[cls] / (per_launch_ms[cls] * 1e-3) / 1e12
+        tr = TRAFFIC.get(cls)
+        r = {"kernel": cls, "bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_peak,
+             "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
+             "peak_kind": f"bf16 {'burst' if use_burst else 'sustained'} ({peaks['source']}; {why})",
+             "frac_vs_burst": round(achieved / peaks["bf16_tflops"], 4),
+             "frac_vs_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+             "traffic": tr["bytes"] if tr and tr["sha"] == kernel_source_sha() else None,
+             "algorithmic_per_launch": flops_per_launch[cls],
+             "note": ("one launch = the three weight gradients" if cls == "bwd_grad_w" else
+                      "time per call includes the 2-bit code expansion kernel (~14 us); traffic is the GEMM's")}
         if "bf16_tflops" in probe:
-            roof["frac_vs_tcgen05_probe"] = round(achieved / probe["bf16_tflops"], 4)
-    else:
-        roof = {"kernel": dominant, "bound": "unknown"}
+            r["frac_vs_tcgen05_probe"] = round(achieved / probe["bf16_tflops"], 4)
+        return r
+
+    # The dominant kernel: the grouped grad_W GEMM, the largest single kernel of the step
+    # by time (launch list: 38 % of kernel time, the grad_X GEMM 36 %); the grad_X product
+    # is reported beside it.
+    roof = gemm_roofline("bwd_grad_w")
+    roof_gx = gemm_roofline("bwd_grad_x")
     # INT8: no measured peak in the driver's file; derived as 2 x the bf16 rate chosen above (the
     # nominal int8 / bf16 ratio of B200), with this run's tcgen05 probe beside it
     int8_peak = 2 * bf16_peak
@@ -500,6 +515,7 @@ def run_ours(args) -> None:
         "speedup_vs_8_8": round(ms_dense / ms_step, 4),
         "ms_per_step_8_8": round(ms_dense, 4),
         "roofline": roof,
+        "roofline_grad_x": roof_gx,
         "e2e": {"value": round(job_tokens_per_s(ms_e2e, world), 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 3), "steps": e2e_steps,
                 "copies": "pinned host <-> device on separate H2D / D2H streams, overlapped with compute (2 I/O sets)"},
@@ -689,6 +705,10 @@ def run_case(args) -> None:
     hist = torch.empty((19,), dtype=torch.int64, device=dev)
     g_w = (bf(synth.activation_bf16(14, n_out, k_in, std=1e-2, outliers=False)) if args.case == "sgd_quant_mask"
            else None)
+    gw_group = ([{"dy": bf(synth.activation_bf16(15 + i, t, n, std=1e-2, outliers=False)),
+                  "x": bf(synth.activation_bf16(18 + i, t, k)),
+                  "grad_w": torch.empty((n, k), dtype=torch.bfloat16, device=dev)} for i, (_, k, n) in enumerate(LINEARS)]
+                if args.case == "grad_w_grouped" else None)
     flops = 2.0 * t * k_in * n_out
     cases = {
         # algorithmic bytes: W read once (4 B/w), int8 codes, packed codes and mask written
@@ -708,6 +728,9 @@ def run_case(args) -> None:
         "grad_x": (lambda: B.bitlinear_bwd(dy, None, qm["codes"], qm["w_scale"], want_grad_w=False, grad_x=gx,
                                            workspace=ws, k_in=k_in), "TFLOP/s", flops),
         "grad_w": (lambda: B.bitlinear_bwd(dy, x, None, None, want_grad_x=False, grad_w=gw), "TFLOP/s", flops),
+        # the three weight gradients of the 3B MLP (gate, up, down) over t tokens, one launch
+        "grad_w_grouped": (lambda: B.bitlinear_grad_w_grouped(gw_group), "TFLOP/s",
+                           sum(2.0 * t * k * n for _, k, n in LINEARS)),
         # int8-dY input gradient (an approximation; dY quantised per token): dense-equivalent ops
         "grad_x_i8": (lambda: B.bitlinear_grad_x_i8(dy, qm["codes"], qm["w_scale"], k_in=k_in, grad_x=gx,
                                                     workspace=ws_i8), "TOP/s", flops),
@@ -954,6 +977,7 @@ def main(argv=None) -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the N:M sweep and decode sub-records")
     ap.add_argument("--case", choices=["quant_mask", "sgd_quant_mask", "act_quant", "fwd", "fwd_sp", "fwd_codes", "grad_x", "grad_w",
+                                       "grad_w_grouped",
                                        "grad_x_i8", "mask_hist", "mma_peak_i8", "mma_peak_bf16", "mma_peak_sp_i8"],
                     help="time one kernel class alone on the --case-t/k/n shape")
     ap.add_argument("--case-t", type=int, default=TOKENS)

@@ -261,6 +261,32 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const int8_t* xq,
                         uint16_t* grad_x, void* grad_w, int grad_w_dtype, int flags, void* workspace,
                         size_t workspace_bytes, void* stream);
 
+/* One weight gradient of a group (see bitlinear_grad_w_grouped). */
+typedef struct {
+  const uint16_t* dy;  /* [t, n_out] bf16, in: gradient of this linear's output */
+  const uint16_t* x;   /* [t, k_in] bf16, in: this linear's input */
+  int64_t k_in, n_out;
+  void* grad_w;        /* [n_out, k_in], out: bf16 (BL_OUT_BF16) or fp32 (BL_OUT_F32) */
+  int grad_w_dtype;
+} bl_grad_w_problem;
+
+/*
+ * Step a6 for several linears over the same t tokens (e.g. the gate, up and down
+ * projections of an MLP block) in one launch: for each problem, grad_W = dY^T X exactly
+ * as bitlinear_bwd computes it with grad_x = NULL and flags = 0 (the layer's bf16 input,
+ * every latent weight including the masked ones; Sparse-BitNet article, sections 三 and
+ * 六). The products' output tiles are scheduled together, so the partial last wave of
+ * one product is filled with tiles of the next.
+ *
+ *   problems   count entries, 1 <= count <= 4; every pointer 16-byte aligned; shapes
+ *              as bitlinear_bwd (k_in, n_out multiples of 64 and 16); outputs must not
+ *              overlap each other or any input.
+ *   t          tokens, shared by all problems (t = 0 zeroes every grad_w).
+ *
+ * Problems with n_out <= 128 (outside the two-SM tiles) run one after another instead.
+ */
+bl_status bitlinear_grad_w_grouped(const bl_grad_w_problem* problems, int count, int64_t t, void* stream);
+
 /* Bytes of workspace bitlinear_grad_x_i8 needs (0 for an empty problem). */
 size_t bitlinear_grad_x_i8_workspace_size(int64_t t, int64_t k_in, int64_t n_out);
 

@@ -22,5 +22,6 @@ from .bitlinear import (  # noqa: F401
     bitlinear_quant_mask_status,
     bitlinear_quant_mask_workspace_size,
     bitlinear_sgd_quant_mask,
+    bitlinear_grad_w_grouped,
     sp_meta_shape,
 )

@@ -35,6 +35,12 @@ class BlFwdProblem(ctypes.Structure):
                 ("n_out", ctypes.c_int64), ("acc_out", ctypes.c_void_p), ("y_out", ctypes.c_void_p)]
 
 
+class BlGradWProblem(ctypes.Structure):
+    """bl_grad_w_problem of include/bitlinear.h."""
+    _fields_ = [("dy", ctypes.c_void_p), ("x", ctypes.c_void_p), ("k_in", ctypes.c_int64), ("n_out", ctypes.c_int64),
+                ("grad_w", ctypes.c_void_p), ("grad_w_dtype", ctypes.c_int)]
+
+
 # name -> (restype, argtypes), in the order of include/bitlinear.h
 SIGNATURES = {
     "bitlinear_quant_mask_workspace_size": (_SZ, [_I64, _I64]),
@@ -47,6 +53,7 @@ SIGNATURES = {
     "bitlinear_fwd_grouped": (_INT, [_c.POINTER(BlFwdProblem), _INT, _INT, _P]),
     "bitlinear_bwd_workspace_size": (_SZ, [_I64, _I64, _I64, _INT, _INT]),
     "bitlinear_bwd": (_INT, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _INT, _P, _SZ, _P]),
+    "bitlinear_grad_w_grouped": (_INT, [_P, _INT, _I64, _P]),
     "bitlinear_grad_x_i8_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_grad_x_i8": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "bitlinear_mask_threshold_hist": (_INT, [_P, _P, _P, _I64, _I64, _INT, _P, _P]),

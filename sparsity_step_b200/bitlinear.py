@@ -275,6 +275,38 @@ def bitlinear_fwd_grouped(problems: list[dict], *, y_dtype=torch.bfloat16, strea
     return out
 
 
+def bitlinear_grad_w_grouped(problems: list[dict], *, grad_w_dtype=torch.bfloat16, stream=None) -> list[torch.Tensor]:
+    """grad_W = dY^T X of several linears over the same tokens in one launch.
+
+    Each problem is a dict with ``dy`` (bf16 [t, n_out]), ``x`` (bf16 [t, k_in]) and
+    optionally ``grad_w`` (allocated here when missing). Returns the grad_w tensors.
+    """
+    if not 1 <= len(problems) <= 4:
+        raise ValueError("1 to 4 problems")
+    arr = (_lib.BlGradWProblem * len(problems))()
+    out = []
+    t = problems[0]["dy"].shape[0]
+    dev = problems[0]["dy"].device
+    for i, p in enumerate(problems):
+        dy, x = p["dy"], p["x"]
+        _need(dy, torch.bfloat16, None, f"problem {i} dy", dev)
+        n_out = dy.shape[1]
+        if dy.shape[0] != t:
+            raise ValueError(f"problem {i}: every problem needs the same token count ({t})")
+        _need(x, torch.bfloat16, (t, x.shape[1]), f"problem {i} x", dev)
+        k_in = x.shape[1]
+        gw = p.get("grad_w")
+        if gw is None:
+            gw = torch.empty((n_out, k_in), dtype=grad_w_dtype, device=dev)
+        _need(gw, grad_w_dtype, (n_out, k_in), f"problem {i} grad_w", dev)
+        arr[i] = _lib.BlGradWProblem(_ptr(dy), _ptr(x), k_in, n_out, _ptr(gw),
+                                     BL_OUT_F32 if grad_w_dtype == torch.float32 else BL_OUT_BF16)
+        out.append(gw)
+    st = lib().bitlinear_grad_w_grouped(arr, len(problems), t, _stream(stream))
+    check(st, "bitlinear_grad_w_grouped")
+    return out
+
+
 BL_GRADW_DEQUANT_X = 1   # grad_W against the dequantised activations q * a / 127
 
 

@@ -119,8 +119,7 @@ bl_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
 // (g.num_m_blocks / g.num_n_blocks count 256-wide blocks). Sets *launched to false and
 // launches nothing when no CTA pair fits on the device, so the caller can fall back.
 template <bool kI8, bool kAMN, bool kBMN, int kEpi>
-bl_status launch_gemm2(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout, const bl::GemmArgs& g,
-                       cudaStream_t st, bool* launched) {
+bl_status launch_gemm2(const bl::GemmGroup2& G, cudaStream_t st, bool* launched) {
   *launched = false;
   auto kern = bl::gemm_tc2_kernel<kI8, kAMN, kBMN, kEpi>;
   constexpr size_t smem = bl::gemm2_smem_bytes();
@@ -146,13 +145,27 @@ bl_status launch_gemm2(const CUtensorMap& ta, const CUtensorMap& tb, const CUten
     max_clusters = n;
   }
   if (max_clusters <= 0) return BL_OK;
-  const int tiles = g.num_m_blocks * g.num_n_blocks;
+  const int tiles = G.total_tiles;
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
   cfg.gridDim = dim3(2 * clusters);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tout, g);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, G);
   if (e != cudaSuccess) return cuda_fail(e, "gemm2 launch");
   *launched = true;
   return BL_OK;
+}
+
+// A product as a group of one for the pair kernel (g counts 256-wide blocks).
+bl::GemmGroup2 one_problem(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout, const bl::GemmArgs& g) {
+  bl::GemmGroup2 G{};
+  G.p[0].tmA = ta;
+  G.p[0].tmB = tb;
+  G.p[0].tmOut = tout;
+  G.p[0].g = g;
+  G.p[0].tile_begin = 0;
+  G.count = 1;
+  G.total_tiles = g.num_m_blocks * g.num_n_blocks;
+  G.num_k_blocks = g.num_k_blocks;
+  return G;
 }
 
 // Pairs pay off once the output has at least two 128-row blocks; a single block would
@@ -579,7 +592,8 @@ bl_status enqueue_fwd_i8(const int8_t* xq, const float* absmax, const int8_t* w_
     bl::GemmArgs g2 = g;
     g2.num_m_blocks = static_cast<int>((t + 255) / 256);
     bool launched = false;
-    if (bl_status s = launch_gemm2<true, false, false, bl::EPI_FWD>(ta, tb2, to, g2, st, &launched)) return s;
+    if (bl_status s = launch_gemm2<true, false, false, bl::EPI_FWD>(one_problem(ta, tb2, to, g2), st, &launched))
+      return s;
     if (launched) return BL_OK;
   }
   return launch_gemm<true, false, false, bl::EPI_FWD, true>(ta, tb, to, g, st);
@@ -867,7 +881,8 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const int8_t* xq,
     if (use_cta_pair(t)) {
       bl::GemmArgs g2 = g;
       g2.num_m_blocks = static_cast<int>((t + 255) / 256);
-      if (bl_status s = launch_gemm2<false, false, true, bl::EPI_GRADX>(ta, tb, to, g2, st, &launched)) return s;
+      if (bl_status s = launch_gemm2<false, false, true, bl::EPI_GRADX>(one_problem(ta, tb, to, g2), st, &launched))
+        return s;
     }
     if (!launched)
       if (bl_status s = launch_gemm<false, false, true, bl::EPI_GRADX, true>(ta, tb, to, g, st)) return s;
@@ -906,10 +921,73 @@ bl_status bitlinear_bwd(const uint16_t* dy, const uint16_t* x, const int8_t* xq,
     if (use_cta_pair(n_out)) {
       bl::GemmArgs g2 = g;
       g2.num_m_blocks = static_cast<int>((n_out + 255) / 256);
-      if (bl_status s = launch_gemm2<false, true, true, bl::EPI_GRADW>(ta, tb, to, g2, st, &launched)) return s;
+      if (bl_status s = launch_gemm2<false, true, true, bl::EPI_GRADW>(one_problem(ta, tb, to, g2), st, &launched))
+        return s;
     }
     if (!launched)
       if (bl_status s = launch_gemm<false, true, true, bl::EPI_GRADW, true>(ta, tb, to, g, st)) return s;
+  }
+  return BL_OK;
+}
+
+bl_status bitlinear_grad_w_grouped(const bl_grad_w_problem* problems, int count, int64_t t, void* stream) {
+  g_err[0] = 0;
+  if (!problems || count < 1 || count > bl::kMaxGemmGroup)
+    return fail(BL_ERR_INVALID_ARG, "need 1 to %d problems", bl::kMaxGemmGroup);
+  for (int i = 0; i < count; ++i) {
+    const bl_grad_w_problem& q = problems[i];
+    if (!q.grad_w) return fail(BL_ERR_INVALID_ARG, "problem %d: grad_w is required", i);
+    if ((!q.dy || !q.x) && t != 0) return fail(BL_ERR_INVALID_ARG, "problem %d: dy and x are required", i);
+    if (q.grad_w_dtype != BL_OUT_BF16 && q.grad_w_dtype != BL_OUT_F32)
+      return fail(BL_ERR_INVALID_ARG, "problem %d: grad_w_dtype must be BL_OUT_BF16 or BL_OUT_F32", i);
+    if (bl_status s = check_shape(t, q.k_in, q.n_out)) return s;
+    if ((q.dy && !aligned16(q.dy)) || (q.x && !aligned16(q.x)) || !aligned16(q.grad_w))
+      return fail(BL_ERR_ALIGNMENT, "every pointer must be 16-byte aligned");
+  }
+  cudaStream_t st = as_stream(stream);
+  bool pairs = count > 1 && t > 0;
+  for (int i = 0; i < count; ++i) pairs = pairs && use_cta_pair(problems[i].n_out);
+  if (!pairs) {   // one product at a time (single problem, empty batch or narrow outputs)
+    for (int i = 0; i < count; ++i) {
+      const bl_grad_w_problem& q = problems[i];
+      if (bl_status s = bitlinear_bwd(q.dy, q.x, nullptr, nullptr, nullptr, nullptr, t, q.k_in, q.n_out, nullptr,
+                                      q.grad_w, q.grad_w_dtype, 0, nullptr, 0, stream))
+        return s;
+    }
+    return BL_OK;
+  }
+  bl::GemmGroup2 G{};
+  int tiles = 0;
+  for (int i = 0; i < count; ++i) {
+    const bl_grad_w_problem& q = problems[i];
+    bl::GemmProblem2& P = G.p[i];
+    // A = dY^T: dY [t, n_out] read MN-major (reduction over t); B = X [t, k_in], MN-major
+    if (bl_status s = make_map(&P.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.dy, q.n_out, t, 64, 64)) return s;
+    if (bl_status s = make_map(&P.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.x, q.k_in, t, 64, 64)) return s;
+    bl::GemmArgs& g = P.g;
+    g.M = static_cast<int>(q.n_out);
+    g.N = static_cast<int>(q.k_in);
+    g.num_k_blocks = static_cast<int>((t + 63) / 64);
+    g.num_m_blocks = static_cast<int>((q.n_out + 255) / 256);
+    g.num_n_blocks = static_cast<int>((q.k_in + bl::kBN - 1) / bl::kBN);
+    g.out = q.grad_w;
+    g.out_f32 = q.grad_w_dtype == BL_OUT_F32;
+    set_raster(g, 2.0 * double(q.n_out) * double(t), 2.0 * double(t) * double(q.k_in));
+    if (bl_status s = make_out_map(&P.tmOut, q.grad_w, q.n_out, q.k_in, g.out_f32)) return s;
+    P.tile_begin = tiles;
+    tiles += g.num_m_blocks * g.num_n_blocks;
+  }
+  G.count = count;
+  G.total_tiles = tiles;
+  G.num_k_blocks = static_cast<int>((t + 63) / 64);
+  bool launched = false;
+  if (bl_status s = launch_gemm2<false, true, true, bl::EPI_GRADW>(G, st, &launched)) return s;
+  if (launched) return BL_OK;
+  for (int i = 0; i < count; ++i) {   // no CTA pair fits on this device: one at a time
+    const bl_grad_w_problem& q = problems[i];
+    if (bl_status s = bitlinear_bwd(q.dy, q.x, nullptr, nullptr, nullptr, nullptr, t, q.k_in, q.n_out, nullptr,
+                                    q.grad_w, q.grad_w_dtype, 0, nullptr, 0, stream))
+      return s;
   }
   return BL_OK;
 }

@@ -100,10 +100,34 @@ __device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t adesc, 
       : "memory");
 }
 
+// One launch may run several products of the same kind and the same K (e.g. the grad_W
+// of every linear of an MLP over one token batch): their 256 x 256 tiles are numbered
+// consecutively (problem i owns tiles [tile_begin, tile_begin + m blocks * n blocks))
+// and the pairs stride over the concatenated list, so the last wave of one product no
+// longer leaves pairs idle. A single product is a group of one.
+constexpr int kMaxGemmGroup = 4;
+struct GemmProblem2 {
+  CUtensorMap tmA, tmB, tmOut;
+  GemmArgs g;
+  int tile_begin;
+};
+struct GemmGroup2 {
+  GemmProblem2 p[kMaxGemmGroup];
+  int count;
+  int total_tiles;
+  int num_k_blocks;   // the same for every problem of the group
+};
+// Problem of a tile in the concatenated list (tile_begin ascending).
+__device__ __forceinline__ int group_problem(const GemmGroup2& G, int tile) {
+  int i = 0;
+#pragma unroll
+  for (int j = 1; j < kMaxGemmGroup; ++j) i += (j < G.count && tile >= G.p[j].tile_begin) ? 1 : 0;
+  return i;
+}
+
 template <bool kI8, bool kAMN, bool kBMN, int kEpi>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmOut, const GemmArgs g) {
+    gemm_tc2_kernel(const __grid_constant__ GemmGroup2 G) {
   static_assert(!(kI8 && (kAMN || kBMN)), "the int8 product uses K-major operands only");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -134,9 +158,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    tma_prefetch_desc(&tmOut);
+    for (int i = 0; i < G.count; ++i) {
+      tma_prefetch_desc(&G.p[i].tmA);
+      tma_prefetch_desc(&G.p[i].tmB);
+      tma_prefetch_desc(&G.p[i].tmOut);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
@@ -147,7 +173,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t peer_abort = map_to_rank(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
-  const int num_tiles = g.num_m_blocks * g.num_n_blocks;   // 256 x 256 tiles
+  const int num_tiles = G.total_tiles;   // 256 x 256 tiles of every problem
+  const int num_k_blocks = G.num_k_blocks;
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
 
   if (warp == 0) {
@@ -160,12 +187,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       int local = 0;
       for (int tile = cluster; tile < num_tiles && ok; tile += nclusters, ++local) {
+        const GemmProblem2& P = G.p[group_problem(G, tile)];
         int mb, nb;
-        tile_coords(g, tile, mb, nb);
+        tile_coords(P.g, tile - P.tile_begin, mb, nb);
         const int m0 = mb * 256 + 128 * static_cast<int>(rank);
         const int n0 = nb * 256 + 128 * static_cast<int>(rank);
-        for (int kq = 0; kq < g.num_k_blocks; ++kq) {
-          const int kb = (local & 1) ? g.num_k_blocks - 1 - kq : kq;   // serpentine K order
+        const CUtensorMap* tmA = &P.tmA;
+        const CUtensorMap* tmB = &P.tmB;
+        for (int kq = 0; kq < num_k_blocks; ++kq) {
+          const int kb = (local & 1) ? num_k_blocks - 1 - kq : kq;   // serpentine K order
           if (!mbar_wait(empty0 + 8u * s, ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -175,16 +205,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t a_dst = sA + s * kAHalfBytes, b_dst = sB + s * kBHalfBytes;
           const int kc = kI8 ? kb * 128 : kb * 64;
           if (kAMN) {
-            tma_load_2d_pair(a_dst, &tmA, fb, m0, kc);
-            tma_load_2d_pair(a_dst + 8192, &tmA, fb, m0 + 64, kc);
+            tma_load_2d_pair(a_dst, tmA, fb, m0, kc);
+            tma_load_2d_pair(a_dst + 8192, tmA, fb, m0 + 64, kc);
           } else {
-            tma_load_2d_pair(a_dst, &tmA, fb, kc, m0);
+            tma_load_2d_pair(a_dst, tmA, fb, kc, m0);
           }
           if (kBMN) {
-            tma_load_2d_pair(b_dst, &tmB, fb, n0, kc);
-            tma_load_2d_pair(b_dst + 8192, &tmB, fb, n0 + 64, kc);
+            tma_load_2d_pair(b_dst, tmB, fb, n0, kc);
+            tma_load_2d_pair(b_dst + 8192, tmB, fb, n0 + 64, kc);
           } else {
-            tma_load_2d_pair(b_dst, &tmB, fb, kc, n0);
+            tma_load_2d_pair(b_dst, tmB, fb, kc, n0);
           }
           ++issued;
           if (++s == kStages2) {
@@ -222,7 +252,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
-        for (int kb = 0; kb < g.num_k_blocks; ++kb) {
+        for (int kb = 0; kb < num_k_blocks; ++kb) {
           if (!mbar_wait(full0 + 8u * s, ph, abort_flag)) {
             ok = false;
             break;
@@ -259,7 +289,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quad = warp & 3;
     const int col_begin = (e >> 2) * (kBN / 2);
     const int row_in_tile = 128 * static_cast<int>(rank) + quad * 32 + lane;
-    const float gamma = (kEpi == EPI_GRADW) ? 1.0f : *g.w_scale;
     const uint32_t stage_buf = sOut + static_cast<uint32_t>(e * kStageOutBytes);
     const uint32_t tempty_leader0 = map_to_rank(tempty0, 0);
     int cnt = 0;
@@ -268,14 +297,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int tile = cluster; tile < num_tiles; tile += nclusters, ++local) {
       const int buf = local & 1;
       const uint32_t tph = static_cast<uint32_t>(local >> 1) & 1u;
+      const GemmProblem2& P = G.p[group_problem(G, tile)];
       int mb, nb;
-      tile_coords(g, tile, mb, nb);
+      tile_coords(P.g, tile - P.tile_begin, mb, nb);
       const int row = mb * 256 + row_in_tile;
       const int n0 = nb * kBN;
-      const bool row_ok = row < g.M;
+      const bool row_ok = row < P.g.M;
+      const float gamma = (kEpi == EPI_GRADW) ? 1.0f : *P.g.w_scale;
       float rs = 1.0f;
       if (kEpi == EPI_FWD) {
-        if (row_ok) rs = __fmul_rn(__fdiv_rn(g.row_absmax[row], 127.0f), gamma);
+        if (row_ok) rs = __fmul_rn(__fdiv_rn(P.g.row_absmax[row], 127.0f), gamma);
       } else if (kEpi == EPI_GRADX) {
         rs = gamma;
       }
@@ -286,7 +317,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after_sync();
       const uint32_t t_row = tmem_base + static_cast<uint32_t>(buf * kBN) + (static_cast<uint32_t>(quad * 32) << 16);
-      epilogue_tile_tma<kEpi>(g, &tmOut, t_row, stage_buf, cnt, row - lane, n0, col_begin, rs, lane);
+      epilogue_tile_tma<kEpi>(P.g, &P.tmOut, t_row, stage_buf, cnt, row - lane, n0, col_begin, rs, lane);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(tempty_leader0 + 8u * buf);

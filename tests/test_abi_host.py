@@ -76,6 +76,24 @@ def test_sgd_quant_mask_validation(L):
     assert call(BAD, GOOD, 1e-3, 896, 896, 6, 8, GOOD, GOOD, GOOD, None, None, GOOD, GOOD, ws, None) == -3
 
 
+def test_grad_w_grouped_validation(L):
+    def arr(*probs):
+        a = (_lib.BlGradWProblem * max(1, len(probs)))()
+        for i, p in enumerate(probs):
+            a[i] = _lib.BlGradWProblem(*p)
+        return a
+    good = (GOOD, GOOD, 2048, 11008, GOOD, 0)
+    call = L.bitlinear_grad_w_grouped
+    assert call(None, 1, 4096, None) == -1
+    assert call(arr(good), 0, 4096, None) == -1
+    assert call(arr(good, good, good, good, good), 5, 4096, None) == -1
+    assert call(arr(good, (GOOD, GOOD, 2048, 11008, None, 0)), 2, 4096, None) == -1   # no output
+    assert call(arr(good, (None, GOOD, 2048, 11008, GOOD, 0)), 2, 4096, None) == -1   # no dY
+    assert call(arr(good, (GOOD, GOOD, 2048, 11008, GOOD, 7)), 2, 4096, None) == -1   # output dtype
+    assert call(arr(good, (GOOD, GOOD, 2000, 11008, GOOD, 0)), 2, 4096, None) == -2   # k_in % 64
+    assert call(arr(good, (GOOD, BAD, 2048, 11008, GOOD, 0)), 2, 4096, None) == -3    # alignment
+
+
 def test_quant_mask_noalloc_validation(L):
     assert L.bitlinear_quant_mask_noalloc(None, 896, 896, 6, 8, GOOD, GOOD, GOOD, GOOD, None) == -1
     assert L.bitlinear_quant_mask_noalloc(GOOD, 896, 896, 9, 8, GOOD, GOOD, GOOD, GOOD, None) == -1

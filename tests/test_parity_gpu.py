@@ -203,6 +203,47 @@ def test_config4_training_step(idx):
     full_layer(4, idx, 16384, k_in, n_out, 6, 8, bwd=True, paths=("w_i8",), sample=True)
 
 
+@pytest.mark.parametrize("f32", [False, True], ids=["bf16", "f32"])
+@pytest.mark.parametrize("shapes,t", [([(896, 4864), (896, 4864), (4864, 896)], 1000),
+                                      ([(640, 400), (576, 272)], 257),
+                                      ([(256, 1536), (896, 128), (128, 384)], 300)],
+                         ids=["mlp-0.5b", "ragged", "with-narrow"])
+def test_grad_w_grouped(shapes, t, f32):
+    """Several grad_W products in one launch (tiles of all products scheduled together;
+    a group with an output of <= 128 rows runs one product at a time): each against the
+    oracle's dY^T X."""
+    probs, refs = [], []
+    for i, (k_in, n_out) in enumerate(shapes):
+        x = synth.activation_bf16(300 + i, t, k_in)
+        dy = synth.activation_bf16(310 + i, t, n_out, std=1e-2, outliers=False)
+        probs.append({"dy": bits_to_dev_bf16(dy), "x": bits_to_dev_bf16(x)})
+        refs.append(O.grad_w(dy, x))
+    gws = B.bitlinear_grad_w_grouped(probs, grad_w_dtype=torch.float32 if f32 else torch.bfloat16)
+    torch.cuda.synchronize()
+    for i, (gw, ref) in enumerate(zip(gws, refs)):
+        if f32:
+            assert_grad_close(gw.cpu().numpy(), ref, f"grouped grad_w {i} f32", is_bf16=False)
+        else:
+            assert_grad_close(bf16_dev_to_bits(gw), ref, f"grouped grad_w {i}")
+
+
+def test_grad_w_grouped_training_shape():
+    """The three grad_W of the 3B MLP over 16384 tokens in one launch (the bench step's
+    call), sampled rows against the oracle."""
+    t = 16384
+    probs, ins = [], []
+    for i, (_, k_in, n_out) in enumerate(QWEN3B_MLP):
+        x = synth.activation_bf16(320 + i, t, k_in)
+        dy = synth.activation_bf16(330 + i, t, n_out, std=1e-2, outliers=False)
+        probs.append({"dy": bits_to_dev_bf16(dy), "x": bits_to_dev_bf16(x)})
+        ins.append((dy, x, n_out))
+    gws = B.bitlinear_grad_w_grouped(probs)
+    torch.cuda.synchronize()
+    for i, (gw, (dy, x, n_out)) in enumerate(zip(gws, ins)):
+        rows = sample_rows(n_out, 40 + i)
+        assert_grad_close(bf16_dev_to_bits(gw)[rows], O.grad_w(dy, x, rows=rows), f"grouped grad_w {i}")
+
+
 QWEN3B_LAYER = [("q", 2048, 2048), ("k", 2048, 256), ("v", 2048, 256), ("o", 2048, 2048),
                 ("gate", 2048, 11008), ("up", 2048, 11008), ("down", 11008, 2048)]
 
