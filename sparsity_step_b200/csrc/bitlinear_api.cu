@@ -195,13 +195,13 @@ void set_raster(bl::GemmArgs& g, double a_bytes, double b_bytes) {
 // where the table does not fit gets BL_ERR_CUDA from every call, before anything is
 // enqueued, instead of a launch that would leave y unwritten.
 constexpr int kMaxLayoutDevices = 64;
-int g_dec_layout[kMaxLayoutDevices] = {};   // 0 unchecked, 1 fits, -1 does not fit
-unsigned int g_dec_base_seen[kMaxLayoutDevices] = {};
 std::mutex g_dec_layout_mu;
 
-template <int NG>
+template <int NG, int RB>
 bl_status check_decode_layout(cudaStream_t st) {
-  using C = bl::DecCfg<NG>;
+  using C = bl::DecCfg<NG, RB>;
+  static int g_dec_layout[kMaxLayoutDevices] = {};   // per kernel: 0 unchecked, 1 fits, -1 does not fit
+  static unsigned int g_dec_base_seen[kMaxLayoutDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -214,14 +214,15 @@ bl_status check_decode_layout(cudaStream_t st) {
     if (cap != cudaStreamCaptureStatusNone)
       return fail(BL_ERR_CUDA, "the first decode-kernel call on a device checks its shared-memory layout "
                                "synchronously: make it before stream capture");
-    e = cudaFuncSetAttribute(bl::fwd_codes_mma_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    e = cudaFuncSetAttribute(bl::fwd_codes_mma_kernel<NG, RB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
     static thread_local bl::FwdGroup probe;   // ~16 KB: kept off the stack
     probe.count = 0;
     probe.total_tasks = 0;
     probe.y_f32 = 0;
     probe.layout_probe = 1;
-    bl::fwd_codes_mma_kernel<NG><<<1, C::kThreads, C::kSmemBytes, st>>>(probe);
+    bl::fwd_codes_mma_kernel<NG, RB><<<1, C::kThreads, C::kSmemBytes, st>>>(probe);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "decode layout probe launch");
     e = cudaStreamSynchronize(st);
@@ -239,14 +240,14 @@ bl_status check_decode_layout(cudaStream_t st) {
   return BL_OK;
 }
 
-template <int NG>
+template <int NG, int RB>
 bl_status launch_fwd_codes_ng(const bl::FwdGroup& grp, cudaStream_t st) {
-  using C = bl::DecCfg<NG>;
-  if (bl_status s = check_decode_layout<NG>(st)) return s;
+  using C = bl::DecCfg<NG, RB>;
+  if (bl_status s = check_decode_layout<NG, RB>(st)) return s;
   int64_t blocks = (static_cast<int64_t>(grp.total_tasks) + C::kWarps - 1) / C::kWarps;
   const int64_t cap = int64_t(device_sm_count());   // one CTA per SM (persistent)
   if (blocks > cap) blocks = cap;
-  bl::fwd_codes_mma_kernel<NG><<<static_cast<unsigned>(blocks), C::kThreads, C::kSmemBytes, st>>>(grp);
+  bl::fwd_codes_mma_kernel<NG, RB><<<static_cast<unsigned>(blocks), C::kThreads, C::kSmemBytes, st>>>(grp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return BL_OK;
@@ -308,6 +309,10 @@ bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32
   if (tmax >= kCodesTcMinTokens) return launch_fwd_codes_tc(problems, count, y_f32, st);
   constexpr int ng = 1;   // batches of 9+ tokens took the tensor-core path above
   static thread_local bl::FwdGroup grp;   // ~16 KB: kept off the stack
+  // tasks of two 16-row blocks when every problem's rows split into 32-row blocks
+  bool rb2 = true;
+  for (int i = 0; i < count; ++i) rb2 = rb2 && (problems[i].t == 0 || problems[i].n_out % 32 == 0);
+  const int rows = rb2 ? 32 : 16;
   int64_t tasks = 0;
   int n = 0;
   for (int i = 0; i < count; ++i) {
@@ -324,14 +329,14 @@ bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32
     d.k_in = static_cast<int>(q.k_in);
     d.n_out = static_cast<int>(q.n_out);
     d.task_begin = static_cast<int>(tasks);
-    tasks += (q.n_out / 16) * ((q.t + 8 * ng - 1) / (8 * ng));
+    tasks += (q.n_out / rows) * ((q.t + 8 * ng - 1) / (8 * ng));
     if (tasks > INT32_MAX) return fail(BL_ERR_UNSUPPORTED_SHAPE, "too much work in one call");
   }
   grp.count = n;
   grp.total_tasks = static_cast<int>(tasks);
   grp.y_f32 = y_f32 ? 1 : 0;
   grp.layout_probe = 0;
-  return launch_fwd_codes_ng<ng>(grp, st);
+  return rb2 ? launch_fwd_codes_ng<ng, 2>(grp, st) : launch_fwd_codes_ng<ng, 1>(grp, st);
 }
 
 // ------------------------------------------------------------------ quant_mask launches

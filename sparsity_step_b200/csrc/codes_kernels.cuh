@@ -198,23 +198,26 @@ __device__ __forceinline__ void decode_chunk(DecAcc<NG>& acc, uint32_t lanesel, 
 // the table; slots 1.. sit above it, from kDecHighBase.
 constexpr int kDecDepth = 4;
 
-template <int NG>
+// RB = 16-row blocks per task: a task of RB blocks shares each chunk's activations and the
+// ring bookkeeping between RB x 8 MMAs (RB = 2 with half the warps keeps the ring's bytes).
+template <int NG, int RB = 1>
 struct DecCfg {
-  static constexpr int kWarps = NG == 1 ? 32 : 16;
+  static constexpr int kWarps = (NG == 1 ? 32 : 16) / RB;
   static constexpr int kThreads = kWarps * 32;
-  static constexpr uint32_t kSlotBytes = 2u * kThreads * 16u;
+  static constexpr uint32_t kSlotBytes = 2u * RB * kThreads * 16u;
   // enough for any start address of the dynamic shared memory: the last slot ends at
   // kDecHighBase + (kDecDepth - 1) * kSlotBytes
   static constexpr int kSmemBytes = static_cast<int>(kDecHighBase + (kDecDepth - 1) * kSlotBytes);
 };
 static_assert(DecCfg<1>::kSmemBytes <= 232448, "decode ring and table exceed the shared memory of a CTA");
+static_assert(DecCfg<1, 2>::kSmemBytes <= 232448, "decode ring and table exceed the shared memory of a CTA");
 
 struct DecTask {
   const FwdProblem* P;
   int n0, t0, nch;   // first row, first token, chunks of 256 weights
 };
 
-__device__ __forceinline__ DecTask dec_task(const FwdGroup& G, int task, int tok_per_task) {
+__device__ __forceinline__ DecTask dec_task(const FwdGroup& G, int task, int tok_per_task, int rows_per_task) {
   int lo = 0, hi = G.count - 1;   // last problem with task_begin <= task
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -222,19 +225,19 @@ __device__ __forceinline__ DecTask dec_task(const FwdGroup& G, int task, int tok
     else hi = mid - 1;
   }
   const FwdProblem& P = G.p[lo];
-  const int row_blocks = P.n_out >> 4;
+  const int row_blocks = P.n_out / rows_per_task;
   const int local = task - P.task_begin;
   DecTask d;
   d.P = &P;
-  d.n0 = (local % row_blocks) * 16;
+  d.n0 = (local % row_blocks) * rows_per_task;
   d.t0 = (local / row_blocks) * tok_per_task;
   d.nch = (P.k_in + 255) >> 8;
   return d;
 }
 
-template <int NG>   // token groups of 8 per task
-__global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(const __grid_constant__ FwdGroup G) {
-  using C = DecCfg<NG>;
+template <int NG, int RB>   // token groups of 8 and 16-row blocks per task
+__global__ void __launch_bounds__(DecCfg<NG, RB>::kThreads, 1) fwd_codes_mma_kernel(const __grid_constant__ FwdGroup G) {
+  using C = DecCfg<NG, RB>;
   extern __shared__ __align__(1024) uint8_t dsmem[];
   const uint32_t base = smem_u32(dsmem);
   if (G.layout_probe) {
@@ -257,7 +260,8 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(kDecLutAddr + 256u * e + 4u * l), "r"(word) : "memory");
   }
   __syncthreads();
-  constexpr uint32_t kHalf = C::kThreads * 16;   // row g -> row g+8 within a slot
+  // slot layout [segment][thread][16 B]: segment 2b + h holds row 16b + g + 8h of the task
+  constexpr uint32_t kHalf = C::kThreads * 16;
   const uint32_t ring_lo = base + static_cast<uint32_t>(threadIdx.x * 16);
   const uint32_t ring_hi = kDecHighBase - C::kSlotBytes + static_cast<uint32_t>(threadIdx.x * 16);
   auto slot_addr = [&](int s) { return s == 0 ? ring_lo : ring_hi + static_cast<uint32_t>(s) * C::kSlotBytes; };
@@ -276,7 +280,7 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
   bool p_tail_ok = true;            // this thread's part of a partial last chunk is in range
   auto p_start = [&]() {
     if (p_task < G.total_tasks) {
-      const DecTask d = dec_task(G, p_task, tok_per_task);
+      const DecTask d = dec_task(G, p_task, tok_per_task, 16 * RB);
       p_kb = d.P->k_in >> 2;
       p_src = d.P->codes + static_cast<int64_t>(d.n0 + g) * p_kb + tig * 16;
       p_left = d.nch;
@@ -290,8 +294,9 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
     if (p_task < G.total_tasks) {
       const bool valid = p_left > 1 || p_tail_ok;
       const uint32_t dst = slot_addr(issued % kDecDepth);
-      cp_async16(dst, valid ? p_src : G.p[0].codes, valid);
-      cp_async16(dst + kHalf, valid ? p_src + 8 * p_kb : G.p[0].codes, valid);
+#pragma unroll
+      for (int sg = 0; sg < 2 * RB; ++sg)
+        cp_async16(dst + sg * kHalf, valid ? p_src + (16 * (sg >> 1) + 8 * (sg & 1)) * p_kb : G.p[0].codes, valid);
       p_src += 64;
       if (--p_left == 0) {
         p_task += warps;
@@ -306,7 +311,7 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
 
   int consumed = 0;
   for (int task = blockIdx.x * C::kWarps + wid; task < G.total_tasks; task += warps) {
-    const DecTask d = dec_task(G, task, tok_per_task);
+    const DecTask d = dec_task(G, task, tok_per_task, 16 * RB);
     const FwdProblem& P = *d.P;
     const int K = P.k_in;
     const int8_t* xrow[NG];
@@ -315,25 +320,35 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
       const int tok = min(d.t0 + 8 * j + g, P.t - 1);   // past-the-end tokens feed unstored columns
       xrow[j] = P.xq + static_cast<int64_t>(tok) * K + tig * 64;
     }
-    DecAcc<NG> accs;
+    DecAcc<NG> accs[RB];
 #pragma unroll
-    for (int k = 0; k < DecAcc<NG>::kSets; ++k)
+    for (int b = 0; b < RB; ++b)
 #pragma unroll
-      for (int j = 0; j < NG; ++j) accs.v[k][j][0] = accs.v[k][j][1] = accs.v[k][j][2] = accs.v[k][j][3] = 0;
-    auto next_codes = [&](uint4& c0, uint4& c1) {
+      for (int k = 0; k < DecAcc<NG>::kSets; ++k)
+#pragma unroll
+        for (int j = 0; j < NG; ++j)
+          accs[b].v[k][j][0] = accs[b].v[k][j][1] = accs[b].v[k][j][2] = accs[b].v[k][j][3] = 0;
+    // one chunk: this thread's code words of every row block, its activations, 8 MMAs per block
+    auto chunk = [&](const uint4 (&xv)[NG][4]) {
       produce_one();                      // chunk consumed + kDecDepth - 1
       cp_async_wait<kDecDepth - 1>();     // chunk `consumed` has landed (own copies only)
       const uint32_t slot = slot_addr(consumed % kDecDepth);
-      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(c0.x), "=r"(c0.y), "=r"(c0.z), "=r"(c0.w) : "r"(slot));
-      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w)
-                   : "r"(slot + kHalf));
       ++consumed;
+#pragma unroll
+      for (int b = 0; b < RB; ++b) {
+        uint4 c0, c1;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(c0.x), "=r"(c0.y), "=r"(c0.z), "=r"(c0.w) : "r"(slot + 2 * b * kHalf));
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w) : "r"(slot + (2 * b + 1) * kHalf));
+        decode_chunk<NG>(accs[b], lanesel, c0, c1, xv);
+      }
     };
     const int nfull = K >> 8;
     // full chunks: every thread's 64 weights are in range. The chunk's activations are
-    // loaded at its start (L1/L2 hits; the 32 resident warps hide the latency): a
-    // register prefetch of the next chunk's activations measured 5 % slower at batch 1,
-    // from the copies it costs and the registers it holds.
+    // loaded at its start (L1/L2 hits; the resident warps hide the latency): a register
+    // prefetch of the next chunk's activations measured 5 % slower at batch 1, from the
+    // copies it costs and the registers it holds.
     for (int ch = 0; ch < nfull; ++ch) {
       uint4 xv[NG][4];
 #pragma unroll
@@ -342,13 +357,9 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
 #pragma unroll
         for (int q = 0; q < 4; ++q) xv[j][q] = __ldg(xp + q);
       }
-      uint4 c0, c1;
-      next_codes(c0, c1);
-      decode_chunk<NG>(accs, lanesel, c0, c1, xv);
+      chunk(xv);
     }
     if (K & 255) {   // partial last chunk: threads past the end use zero activations
-      uint4 c0, c1;
-      next_codes(c0, c1);
       const bool mine = nfull * 256 + 64 * tig < K;
       uint4 xv[NG][4];
 #pragma unroll
@@ -357,33 +368,30 @@ __global__ void __launch_bounds__(DecCfg<NG>::kThreads, 1) fwd_codes_mma_kernel(
 #pragma unroll
         for (int q = 0; q < 4; ++q) xv[j][q] = mine ? __ldg(xp + q) : zero;
       }
-      decode_chunk<NG>(accs, lanesel, c0, c1, xv);
+      chunk(xv);
     }
-    int acc[NG][4];
-#pragma unroll
-    for (int j = 0; j < NG; ++j)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        int sum = 0;
-#pragma unroll
-        for (int k = 0; k < DecAcc<NG>::kSets; ++k) sum += accs.v[k][j][v];
-        acc[j][v] = sum;
-      }
-    // C fragment: acc[j][0..1] = row g, tokens 2*tig, 2*tig+1; acc[j][2..3] = row g+8
+    // C fragment of block b: acc[j][0..1] = row 16b + g, tokens 2*tig, 2*tig+1;
+    // acc[j][2..3] = row 16b + g + 8
     const float gamma = *P.w_scale;
 #pragma unroll
-    for (int j = 0; j < NG; ++j) {
+    for (int b = 0; b < RB; ++b) {
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const int tok = d.t0 + 8 * j + 2 * tig + (v & 1);
-        const int n = d.n0 + g + ((v >> 1) << 3);
-        if (tok < P.t) {
-          const float rs = __fmul_rn(__fdiv_rn(P.absmax[tok], 127.0f), gamma);
-          const float y = __fmul_rn(static_cast<float>(acc[j][v]), rs);
-          const int64_t off = static_cast<int64_t>(tok) * P.n_out + n;
-          if (G.y_f32) static_cast<float*>(P.y)[off] = y;
-          else static_cast<__nv_bfloat16*>(P.y)[off] = __float2bfloat16_rn(y);
-          if (P.acc != nullptr) P.acc[off] = acc[j][v];
+      for (int j = 0; j < NG; ++j) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          int accv = 0;
+#pragma unroll
+          for (int k = 0; k < DecAcc<NG>::kSets; ++k) accv += accs[b].v[k][j][v];
+          const int tok = d.t0 + 8 * j + 2 * tig + (v & 1);
+          const int n = d.n0 + 16 * b + g + ((v >> 1) << 3);
+          if (tok < P.t) {
+            const float rs = __fmul_rn(__fdiv_rn(P.absmax[tok], 127.0f), gamma);
+            const float y = __fmul_rn(static_cast<float>(accv), rs);
+            const int64_t off = static_cast<int64_t>(tok) * P.n_out + n;
+            if (G.y_f32) static_cast<float*>(P.y)[off] = y;
+            else static_cast<__nv_bfloat16*>(P.y)[off] = __float2bfloat16_rn(y);
+            if (P.acc != nullptr) P.acc[off] = accv;
+          }
         }
       }
     }
