@@ -298,16 +298,13 @@ bl_status launch_fwd_codes_tc(const bl_fwd_problem* problems, int count, bool y_
 
 // Token batches of more than 8 tokens (the largest in a call) take the tensor-core
 // product from codes; up to 8 the warp-MMA kernel (one 8-token MMA column group).
-// Measured on the 36-layer decode stack: 12 tokens 0.526 ms on two warp-MMA column
-// groups against 0.38 ms for 16 tokens on the tensor cores.
+// Measured on the 36-layer decode stack: 12 and 16 tokens on two warp-MMA column groups
+// (32-row tasks) 0.377 and 0.391 ms, on the tensor cores 0.374 and 0.377 ms.
 constexpr int64_t kCodesTcMinTokens = 9;
 
-bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32, cudaStream_t st) {
-  int64_t tmax = 0;
-  for (int i = 0; i < count; ++i) tmax = problems[i].t > tmax ? problems[i].t : tmax;
-  if (tmax == 0) return BL_OK;
-  if (tmax >= kCodesTcMinTokens) return launch_fwd_codes_tc(problems, count, y_f32, st);
-  constexpr int ng = 1;   // batches of 9+ tokens took the tensor-core path above
+// Warp-MMA decode kernel with NG token groups of 8 per task (problems validated).
+template <int NG>
+bl_status launch_fwd_codes_mma(const bl_fwd_problem* problems, int count, bool y_f32, cudaStream_t st) {
   static thread_local bl::FwdGroup grp;   // ~16 KB: kept off the stack
   // tasks of RB 16-row blocks: the largest RB in {2, 1} that divides every problem's rows
   // (measured on B200, 36-layer 3B decode step: RB = 2 0.180 ms at batch 1, RB = 4 with a
@@ -332,14 +329,22 @@ bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32
     d.k_in = static_cast<int>(q.k_in);
     d.n_out = static_cast<int>(q.n_out);
     d.task_begin = static_cast<int>(tasks);
-    tasks += (q.n_out / rows) * ((q.t + 8 * ng - 1) / (8 * ng));
+    tasks += (q.n_out / rows) * ((q.t + 8 * NG - 1) / (8 * NG));
     if (tasks > INT32_MAX) return fail(BL_ERR_UNSUPPORTED_SHAPE, "too much work in one call");
   }
   grp.count = n;
   grp.total_tasks = static_cast<int>(tasks);
   grp.y_f32 = y_f32 ? 1 : 0;
   grp.layout_probe = 0;
-  return rb == 2 ? launch_fwd_codes_ng<ng, 2>(grp, st) : launch_fwd_codes_ng<ng, 1>(grp, st);
+  return rb == 2 ? launch_fwd_codes_ng<NG, 2>(grp, st) : launch_fwd_codes_ng<NG, 1>(grp, st);
+}
+
+bl_status launch_fwd_codes(const bl_fwd_problem* problems, int count, bool y_f32, cudaStream_t st) {
+  int64_t tmax = 0;
+  for (int i = 0; i < count; ++i) tmax = problems[i].t > tmax ? problems[i].t : tmax;
+  if (tmax == 0) return BL_OK;
+  if (tmax >= kCodesTcMinTokens) return launch_fwd_codes_tc(problems, count, y_f32, st);
+  return launch_fwd_codes_mma<1>(problems, count, y_f32, st);
 }
 
 // ------------------------------------------------------------------ quant_mask launches
