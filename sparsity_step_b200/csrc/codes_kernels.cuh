@@ -204,10 +204,11 @@ template <int NG, int RB = 1>
 struct DecCfg {
   static constexpr int kWarps = (NG == 1 ? 32 : 16) / RB;
   static constexpr int kThreads = kWarps * 32;
+  static constexpr int kDepth = kDecDepth;   // ring slots (chunks in flight + 1)
   static constexpr uint32_t kSlotBytes = 2u * RB * kThreads * 16u;
   // enough for any start address of the dynamic shared memory: the last slot ends at
-  // kDecHighBase + (kDecDepth - 1) * kSlotBytes
-  static constexpr int kSmemBytes = static_cast<int>(kDecHighBase + (kDecDepth - 1) * kSlotBytes);
+  // kDecHighBase + (kDepth - 1) * kSlotBytes
+  static constexpr int kSmemBytes = static_cast<int>(kDecHighBase + (kDepth - 1) * kSlotBytes);
 };
 static_assert(DecCfg<1>::kSmemBytes <= 232448, "decode ring and table exceed the shared memory of a CTA");
 static_assert(DecCfg<1, 2>::kSmemBytes <= 232448, "decode ring and table exceed the shared memory of a CTA");
@@ -293,7 +294,7 @@ __global__ void __launch_bounds__(DecCfg<NG, RB>::kThreads, 1) fwd_codes_mma_ker
   auto produce_one = [&]() {   // always commits one group (empty past the end)
     if (p_task < G.total_tasks) {
       const bool valid = p_left > 1 || p_tail_ok;
-      const uint32_t dst = slot_addr(issued % kDecDepth);
+      const uint32_t dst = slot_addr(issued % C::kDepth);
 #pragma unroll
       for (int sg = 0; sg < 2 * RB; ++sg)
         cp_async16(dst + sg * kHalf, valid ? p_src + (16 * (sg >> 1) + 8 * (sg & 1)) * p_kb : G.p[0].codes, valid);
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(DecCfg<NG, RB>::kThreads, 1) fwd_codes_mma_ker
     ++issued;
   };
 #pragma unroll
-  for (int i = 0; i < kDecDepth - 1; ++i) produce_one();
+  for (int i = 0; i < C::kDepth - 1; ++i) produce_one();
 
   int consumed = 0;
   for (int task = blockIdx.x * C::kWarps + wid; task < G.total_tasks; task += warps) {
@@ -330,9 +331,9 @@ __global__ void __launch_bounds__(DecCfg<NG, RB>::kThreads, 1) fwd_codes_mma_ker
           accs[b].v[k][j][0] = accs[b].v[k][j][1] = accs[b].v[k][j][2] = accs[b].v[k][j][3] = 0;
     // one chunk: this thread's code words of every row block, its activations, 8 MMAs per block
     auto chunk = [&](const uint4 (&xv)[NG][4]) {
-      produce_one();                      // chunk consumed + kDecDepth - 1
-      cp_async_wait<kDecDepth - 1>();     // chunk `consumed` has landed (own copies only)
-      const uint32_t slot = slot_addr(consumed % kDecDepth);
+      produce_one();                      // chunk consumed + kDepth - 1
+      cp_async_wait<C::kDepth - 1>();     // chunk `consumed` has landed (own copies only)
+      const uint32_t slot = slot_addr(consumed % C::kDepth);
       ++consumed;
 #pragma unroll
       for (int b = 0; b < RB; ++b) {
