@@ -273,8 +273,14 @@ __global__ void __launch_bounds__(DecCfg<NG, RB>::kThreads, 1) fwd_codes_mma_ker
   const int tok_per_task = 8 * NG;
   const uint4 zero = make_uint4(0, 0, 0, 0);
 
-  // producer cursor: (task, chunk) running kDecDepth - 1 chunks ahead, across tasks
-  int p_task = blockIdx.x * C::kWarps + wid;
+  // Task order: task t runs on CTA t % gridDim.x (one CTA per SM), on its warp
+  // (t / gridDim.x) % kWarps, so consecutive tasks -- neighbouring rows of one product,
+  // of equal cost -- go to different SMs and every SM gets a near-equal share of each
+  // product's work (assigning consecutive tasks to the warps of one CTA left one SM with
+  // up to 3.4x the average work for some layer stacks).
+  const int task0 = blockIdx.x + gridDim.x * wid;
+  // producer cursor: (task, chunk) running kDepth - 1 chunks ahead, across tasks
+  int p_task = task0;
   const uint8_t* p_src = nullptr;   // this thread's 16 code bytes of row n0 + g, next chunk
   int64_t p_kb = 0;                 // code bytes per row
   int p_left = 0;                   // chunks left in the producer's task
@@ -311,7 +317,7 @@ __global__ void __launch_bounds__(DecCfg<NG, RB>::kThreads, 1) fwd_codes_mma_ker
   for (int i = 0; i < C::kDepth - 1; ++i) produce_one();
 
   int consumed = 0;
-  for (int task = blockIdx.x * C::kWarps + wid; task < G.total_tasks; task += warps) {
+  for (int task = task0; task < G.total_tasks; task += warps) {
     const DecTask d = dec_task(G, task, tok_per_task, 16 * RB);
     const FwdProblem& P = *d.P;
     const int K = P.k_in;
