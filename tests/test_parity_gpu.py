@@ -206,8 +206,9 @@ def test_config4_training_step(idx):
 @pytest.mark.parametrize("f32", [False, True], ids=["bf16", "f32"])
 @pytest.mark.parametrize("shapes,t", [([(896, 4864), (896, 4864), (4864, 896)], 1000),
                                       ([(640, 400), (576, 272)], 257),
-                                      ([(256, 1536), (896, 128), (128, 384)], 300)],
-                         ids=["mlp-0.5b", "ragged", "with-narrow"])
+                                      ([(256, 1536), (896, 128), (128, 384)], 300),
+                                      ([(512, 768)], 129)],
+                         ids=["mlp-0.5b", "ragged", "with-narrow", "single"])
 def test_grad_w_grouped(shapes, t, f32):
     """Several grad_W products in one launch (tiles of all products scheduled together;
     a group with an output of <= 128 rows runs one product at a time): each against the
