@@ -3,12 +3,16 @@
 // BitNet b1.58 2B4T article (lsdiaocha.cn), section 一: activations are quantised
 // to 8-bit integers; section 四: W1.58A8 (ternary weights x int8 activations).
 //
-// Each CTA handles R token rows. Each thread loads its 16-byte vectors of the rows
-// once and keeps them in registers; a row's absmax is a block max over |bf16| bit
-// patterns (exact, order-free); then q = clamp(rint(x * (127 / a)), -128, 127) with
-// one IEEE fp32 division per row and one fp32 multiply per element (no FMA), and the
-// int8 rows are written with 8-byte stores. HBM traffic: 2 B read + 1 B written per
-// element, + 4 B per row.
+// Every kernel reads a row once: a row's absmax is a max over |bf16| bit patterns
+// (exact, order-free); then q = clamp(rint(x * (127 / a)), -128, 127) with one IEEE
+// fp32 division per row, one fp32 multiply per element (no FMA) and one saturating
+// round-to-nearest-even conversion, and the int8 rows are written with 8-byte stores.
+// HBM traffic: 2 B read + 1 B written per element, + 4 B per row. By row width:
+//   act_quant_warp_kernel  k_in <= 4096: one warp per row, row in registers;
+//   act_quant_ring_kernel  k_in <= 16384: persistent CTAs streaming their next row into
+//                          a shared-memory ring while quantising the current one;
+//   act_quant_kernel       k_in <= 32768: one CTA per row, row in registers;
+//   act_quant_long_kernel  wider: two reads (max, then quantise).
 #pragma once
 
 #include "common.cuh"
