@@ -344,6 +344,17 @@ def test_codes_at_rounding_boundary():
     check_quant_mask(gpu_quant_mask(w2, 8, 8), ref, "boundary")
 
 
+@pytest.mark.parametrize("k_in", [20480, 32768, 65536], ids=["cta-12", "cta-16", "two-pass"])
+def test_act_quant_wide_rows(k_in):
+    """Rows wider than the ring kernel takes (one CTA per row with 12 or 16 vectors per
+    thread; two reads beyond 32768): bit-exact xq and absmax, a zero row included."""
+    x = synth.activation_bf16(400, 5, k_in)
+    x[2, :] = 0
+    ref_q, ref_a = O.act_quant(x)
+    xq, a = gpu_act_quant(x)
+    check_act_quant(xq, a, ref_q, ref_a, f"wide rows k={k_in}")
+
+
 def test_zero_activation_rows_and_empty_batch():
     x = synth.activation_bf16(88, 6, 896)
     x[2, :] = 0
