@@ -24,10 +24,13 @@ def gpu_quant_mask(w_np, n, m):
     return out
 
 
-def check_quant_mask(out, ref, tag, sp_rows=None):
+def check_quant_mask(out, ref, tag, sp_rows=None, has_mask=True):
     g = out["w_scale"].cpu().numpy()[:1]
     assert_exact(g.view(np.uint32), np.array([ref["gamma"]], np.float32).view(np.uint32), f"{tag} gamma")
-    assert_exact(out["mask"].cpu().numpy(), ref["mask"], f"{tag} mask")
+    if has_mask:
+        assert_exact(out["mask"].cpu().numpy(), ref["mask"], f"{tag} mask")
+    else:
+        assert "mask" not in out, f"{tag}: a mask came back unasked"
     assert_exact(out["codes"].cpu().numpy(), ref["codes_packed"], f"{tag} codes")
     assert_exact(out["w_i8"].cpu().numpy(), ref["mcode"], f"{tag} w_i8")
     if "sp_values" in out:
@@ -327,6 +330,29 @@ def test_mask_ties(nm):
     w[0, :8] = 0.0   # an all-zero group (all ties, gamma still positive)
     ref = O.quant_mask(w, n, m)
     check_quant_mask(gpu_quant_mask(w, n, m), ref, f"ties {n}:{m}")
+
+
+@pytest.mark.parametrize("nm", [(6, 8), (2, 4), (3, 4), (2, 8)], ids=lambda v: f"{v[0]}of{v[1]}")
+def test_quant_mask_without_mask_output(nm):
+    """No mask output wanted: pass 2 ranks the groups itself (the keep bits never reach
+    memory); codes, int8 codes, gamma and, for 2:4-valid masks, the 2:4 form stay exact."""
+    n, m = nm
+    w = synth.latent_weight(410, 272, 896)
+    w[5, 8:16] = w[5, 8]   # a tied group
+    ref = O.quant_mask(w, n, m)
+    out = B.bitlinear_quant_mask(f32_to_dev(w), n, m, want_mask=False, want_sp=n <= 2)
+    torch.cuda.synchronize()
+    assert B.bitlinear_quant_mask_status(out["workspace"]) == 0
+    check_quant_mask(out, ref, f"no mask output {n}:{m}", has_mask=False)
+    # the same with the SGD step fused into pass 1
+    g = synth.activation_bf16(411, 272, 896)
+    ref = O.sgd_quant_mask(w, g, 3e-3, n, m)
+    w_dev = f32_to_dev(w)
+    out = B.bitlinear_sgd_quant_mask(w_dev, bits_to_dev_bf16(g), 3e-3, n, m, want_mask=False, want_sp=n <= 2)
+    torch.cuda.synchronize()
+    assert B.bitlinear_quant_mask_status(out["workspace"]) == 0
+    assert_exact(w_dev.cpu().numpy().view(np.uint32), ref["w"].view(np.uint32), f"sgd {n}:{m} updated W")
+    check_quant_mask(out, ref, f"sgd, no mask output {n}:{m}", has_mask=False)
 
 
 def test_codes_at_rounding_boundary():
