@@ -559,7 +559,7 @@ bl_status enqueue_act_quant(const uint16_t* x, int64_t t, int64_t k_in, int8_t* 
     if (k8 <= 128) bl::act_quant_warp_kernel<4><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
     else if (k8 <= 256) bl::act_quant_warp_kernel<8><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
     else bl::act_quant_warp_kernel<16><<<gb, 256, 0, st>>>(xv, t, k8, xq_out, absmax_out);
-  } else {   // one CTA per row
+  } else {   // up to 16384 wide: persistent ring CTAs; wider: one CTA per row
     const int vpt = (k8 + 255) / 256;
     bl_status s = BL_OK;
     if (vpt <= 4) s = launch_act_quant_ring<4>(xv, t, k8, xq_out, absmax_out, st);
