@@ -1,6 +1,7 @@
 // C ABI of the BitLinear path (declared in include/bitlinear.h): argument checks,
 // workspace layout, TMA descriptor encoding and kernel dispatch. No allocation:
 // the caller owns every buffer.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -36,6 +37,33 @@ bl_status cuda_fail(cudaError_t e, const char* what) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// One-time setup of a kernel on a device: its dynamic shared-memory limit and the
+// occupancy figure the launch sizes its grid by. A kernel attribute belongs to the
+// context of the device that was current when it was set, so a process that drives
+// several devices sets it up once per device. Threads that race on the first call both
+// run the setup (idempotent) and store the same value.
+constexpr int kMaxSetupDevices = 64;
+struct PerDeviceSetup {
+  std::atomic<int> v[kMaxSetupDevices];   // value + 1; 0 = not set up on that device
+};
+
+template <class F>
+bl_status per_device_setup(PerDeviceSetup& c, int* out, F&& setup) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxSetupDevices) return fail(BL_ERR_INVALID_ARG, "device ordinal %d not supported", dev);
+  int v = c.v[dev].load(std::memory_order_acquire);
+  if (v == 0) {
+    int r = 0;
+    if (bl_status s = setup(&r)) return s;
+    v = r + 1;
+    c.v[dev].store(v, std::memory_order_release);
+  }
+  *out = v - 1;
+  return BL_OK;
+}
 
 bl_status check_shape(int64_t t, int64_t k_in, int64_t n_out) {
   if (t < 0 || t > (int64_t(1) << 31) - 1) return fail(BL_ERR_UNSUPPORTED_SHAPE, "t=%lld out of range", (long long)t);
@@ -101,12 +129,15 @@ bl_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
                       cudaStream_t st) {
   auto kern = bl::gemm_tc_kernel<kI8, kAMN, kBMN, kEpi, kTmaStore>;
   constexpr size_t smem = bl::gemm_smem_bytes(kTmaStore);
-  static bool attr_set = false;   // per instantiation; cheap to repeat if raced
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-    attr_set = true;
-  }
+  static PerDeviceSetup setup;   // per instantiation
+  int unused = 0;
+  if (bl_status s = per_device_setup(setup, &unused, [&](int* r) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
+        *r = 1;
+        return BL_OK;
+      }))
+    return s;
   const int tiles = g.num_m_blocks * g.num_n_blocks;
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
   kern<<<grid, bl::kGemmThreads, smem, st>>>(ta, tb, tout, g);
@@ -134,16 +165,20 @@ bl_status launch_gemm2(const bl::GemmGroup2& G, cudaStream_t st, bool* launched)
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  static int max_clusters = -1;   // per instantiation
-  if (max_clusters < 0) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm2)");
-    cfg.gridDim = dim3(2 * (device_sm_count() / 2));
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(gemm2)");
-    max_clusters = n;
-  }
+  static PerDeviceSetup setup;   // per instantiation
+  int max_clusters = 0;
+  if (bl_status s = per_device_setup(setup, &max_clusters, [&](int* r) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm2)");
+        cudaLaunchConfig_t probe = cfg;
+        probe.gridDim = dim3(2 * (device_sm_count() / 2));
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &probe);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(gemm2)");
+        *r = n > 0 ? n : 0;
+        return BL_OK;
+      }))
+    return s;
   if (max_clusters <= 0) return BL_OK;
   const int tiles = G.total_tiles;
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
@@ -282,13 +317,16 @@ bl_status launch_fwd_codes_tc(const bl_fwd_problem* problems, int count, bool y_
   grp.total_tasks = static_cast<int>(tasks);
   grp.y_f32 = y_f32 ? 1 : 0;
   grp.layout_probe = 0;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(bl::fwd_codes_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         bl::kTcSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(codes tc)");
-    attr_set = true;
-  }
+  static PerDeviceSetup setup;
+  int unused = 0;
+  if (bl_status s = per_device_setup(setup, &unused, [&](int* r) {
+        cudaError_t e = cudaFuncSetAttribute(bl::fwd_codes_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             bl::kTcSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(codes tc)");
+        *r = 1;
+        return BL_OK;
+      }))
+    return s;
   const int64_t blocks = tasks < device_sm_count() ? tasks : device_sm_count();
   bl::fwd_codes_tc_kernel<<<static_cast<unsigned>(blocks), bl::kTcThreads, bl::kTcSmemBytes, st>>>(grp);
   cudaError_t e = cudaGetLastError();
@@ -374,15 +412,17 @@ int qm_blocks(int64_t numel);
 int qm_blocks_launch(int64_t numel, int resident);
 
 // Resident 256-thread blocks per SM of a kernel (registers decide it here), looked up
-// once per kernel; 1 if the query fails.
+// once per kernel and device; 1 if the query fails.
 template <typename K>
-int resident_blocks(K kern, int* cache) {
-  if (*cache <= 0) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, bl::kQmThreads, 0) != cudaSuccess || n <= 0) n = 1;
-    *cache = n;
-  }
-  return *cache;
+int resident_blocks(K kern, PerDeviceSetup& cache) {
+  int n = 1;
+  per_device_setup(cache, &n, [&](int* r) {
+    int m = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, kern, bl::kQmThreads, 0) != cudaSuccess || m <= 0) m = 1;
+    *r = m;
+    return BL_OK;
+  });
+  return n > 0 ? n : 1;
 }
 
 // Pass 2 for one compile-time N:M and mask source; the 2:4 form exists only for
@@ -390,7 +430,7 @@ int resident_blocks(K kern, int* cache) {
 template <int M, int NK, bool kMaskIn>
 void launch_codes(const uint4* w4, int64_t n8, int n_keep, float* gamma, const QmOutputs& o, cudaStream_t st) {
   constexpr bool kSpOk = NK <= 2;
-  static int occ = 0, occ_sp = 0;   // per instantiation
+  static PerDeviceSetup occ, occ_sp;   // per instantiation
   auto grid = [&](int resident) {
     const int64_t g = (n8 + bl::kQmThreads - 1) / bl::kQmThreads;
     const int64_t cap = int64_t(device_sm_count()) * resident;
@@ -400,12 +440,12 @@ void launch_codes(const uint4* w4, int64_t n8, int n_keep, float* gamma, const Q
   uint2* w_i8 = reinterpret_cast<uint2*>(o.w_i8);
   if (kSpOk && o.sp_values != nullptr) {
     auto k = bl::qm_codes_kernel<M, NK, kMaskIn, kSpOk>;
-    k<<<grid(resident_blocks(k, &occ_sp)), bl::kQmThreads, 0, st>>>(w4, n8, n_keep, gamma, o.mask, codes, w_i8,
+    k<<<grid(resident_blocks(k, occ_sp)), bl::kQmThreads, 0, st>>>(w4, n8, n_keep, gamma, o.mask, codes, w_i8,
                                                                      reinterpret_cast<uint32_t*>(o.sp_values),
                                                                      o.sp_meta, o.k8, o.meta_pitch);
   } else {
     auto k = bl::qm_codes_kernel<M, NK, kMaskIn, false>;
-    k<<<grid(resident_blocks(k, &occ)), bl::kQmThreads, 0, st>>>(w4, n8, n_keep, gamma, o.mask, codes, w_i8, nullptr,
+    k<<<grid(resident_blocks(k, occ)), bl::kQmThreads, 0, st>>>(w4, n8, n_keep, gamma, o.mask, codes, w_i8, nullptr,
                                                                   nullptr, o.k8, o.meta_pitch);
   }
 }
@@ -414,9 +454,9 @@ void launch_codes(const uint4* w4, int64_t n8, int n_keep, float* gamma, const Q
 template <int M, int NK, bool kMask, bool kUpdate>
 void launch_sum(const uint4* w4, int64_t numel, int n_keep, const QmOutputs& o, const bl::QmScratch& q, float* gamma,
                 const QmUpdate& u, cudaStream_t st) {
-  static int occ = 0;   // per instantiation
+  static PerDeviceSetup occ;   // per instantiation
   auto k = bl::qm_sum_mask_kernel<M, NK, kMask, kUpdate>;
-  const int grid = qm_blocks_launch(numel, device_sm_count() * resident_blocks(k, &occ));
+  const int grid = qm_blocks_launch(numel, device_sm_count() * resident_blocks(k, occ));
   k<<<grid, bl::kQmThreads, 0, st>>>(w4, numel / 8, numel, n_keep, q, gamma, kMask ? o.mask : nullptr,
                                     reinterpret_cast<uint4*>(u.w), reinterpret_cast<const uint4*>(u.grad), u.lr);
 }
@@ -526,18 +566,21 @@ bl_status launch_act_quant_ring(const uint4* xv, int64_t t, int k8, int8_t* xq_o
                                 cudaStream_t st) {
   constexpr int kD = 2;
   constexpr int smem = kD * VPT * 256 * 16;
-  static int occ = 0;   // per instantiation
-  if (occ <= 0) {
-    cudaError_t e = cudaFuncSetAttribute(bl::act_quant_ring_kernel<VPT, kD>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(act_quant ring)");
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bl::act_quant_ring_kernel<VPT, kD>, 256, smem) !=
-            cudaSuccess ||
-        n <= 0)
-      n = 1;
-    occ = n;
-  }
+  static PerDeviceSetup setup;   // per instantiation
+  int occ = 1;
+  if (bl_status s = per_device_setup(setup, &occ, [&](int* r) {
+        cudaError_t e = cudaFuncSetAttribute(bl::act_quant_ring_kernel<VPT, kD>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(act_quant ring)");
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bl::act_quant_ring_kernel<VPT, kD>, 256, smem) !=
+                cudaSuccess ||
+            n <= 0)
+          n = 1;
+        *r = n;
+        return BL_OK;
+      }))
+    return s;
   int64_t grid = int64_t(device_sm_count()) * occ;
   if (grid > t) grid = t;
   bl::act_quant_ring_kernel<VPT, kD><<<static_cast<unsigned>(grid), 256, smem, st>>>(xv, t, k8, xq_out, absmax_out);
@@ -657,16 +700,21 @@ bl_status enqueue_fwd_sp(const int8_t* xq, const float* absmax, const int8_t* sp
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  static int max_clusters = -1;
-  if (max_clusters < 0) {
-    cudaError_t e = cudaFuncSetAttribute(bl::gemm_sp2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(sparse gemm)");
-    cfg.gridDim = dim3(2 * (device_sm_count() / 2));
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, bl::gemm_sp2_kernel, &cfg);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(sparse gemm)");
-    max_clusters = n;
-  }
+  static PerDeviceSetup setup;
+  int max_clusters = 0;
+  if (bl_status s = per_device_setup(setup, &max_clusters, [&](int* r) {
+        cudaError_t e =
+            cudaFuncSetAttribute(bl::gemm_sp2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(sparse gemm)");
+        cudaLaunchConfig_t probe = cfg;
+        probe.gridDim = dim3(2 * (device_sm_count() / 2));
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, bl::gemm_sp2_kernel, &probe);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(sparse gemm)");
+        *r = n > 0 ? n : 0;
+        return BL_OK;
+      }))
+    return s;
   if (max_clusters <= 0) return fail(BL_ERR_CUDA, "no CTA pair of the sparse product fits on this device");
   const int tiles = g.num_row_blocks * g.num_tok_blocks;
   const int clusters = tiles < max_clusters ? tiles : max_clusters;
