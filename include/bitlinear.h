@@ -25,6 +25,10 @@
  *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). Calls only enqueue work and return; results are ready when the
  *     stream reaches them.
+ *   - Devices and threads: a call runs on the calling thread's current device (the
+ *     stream and every pointer must belong to it; device ordinals 0-63). Each kernel
+ *     is set up (shared-memory limit, occupancy) on the first call that uses it on a
+ *     device, so one process may drive several devices, from one thread or several.
  *   - Shapes: k_in % 64 == 0, 64 <= k_in <= 131072, n_out % 16 == 0, n_out >= 16,
  *     t >= 0 (t = 0 is a valid empty batch; the arrays sized by t may then be
  *     NULL). Else BL_ERR_UNSUPPORTED_SHAPE.
