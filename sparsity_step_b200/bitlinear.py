@@ -2,7 +2,8 @@
 
 Argument marshalling only: each function checks dtypes, devices and contiguity,
 allocates missing outputs with torch (device memory is PyTorch's job here), and
-passes raw pointers plus the current CUDA stream to the library. Every step of the
+passes raw pointers plus a CUDA stream of the tensors' device (its current stream
+unless one is given) to the library, with that device current. Every step of the
 computation runs in the library's CUDA kernels; there is no other code path.
 """
 from __future__ import annotations
@@ -15,9 +16,15 @@ from . import _lib
 from ._lib import BL_OUT_BF16, BL_OUT_F32, check, lib
 
 
-def _stream(stream) -> int:
-    s = torch.cuda.current_stream() if stream is None else stream
-    return int(s.cuda_stream)
+def _call(fn, dev: torch.device, stream, *args) -> int:
+    """One library call on the device that holds the tensors: the library works on the
+    calling thread's current device, so that device is made current for the call, and
+    the stream (last argument) is the given one or that device's current stream."""
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {dev}")
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        return int(fn(*args, int(s.cuda_stream)))
 
 
 def _ptr(t) -> int | None:
@@ -108,9 +115,9 @@ def bitlinear_quant_mask(w: torch.Tensor, n_keep: int, m_group: int, *, want_mas
     if workspace is None:
         workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
     _need_bytes(workspace, ws_bytes, "workspace", dev)
-    st = lib().bitlinear_quant_mask(_ptr(w), n_out, k_in, n_keep, m_group, _ptr(o.get("mask")), _ptr(o["codes"]),
-                                    _ptr(o.get("w_i8")), _ptr(o.get("sp_values")), _ptr(o.get("sp_meta")),
-                                    _ptr(o["w_scale"]), _ptr(workspace), workspace.numel(), _stream(stream))
+    st = _call(lib().bitlinear_quant_mask, dev, stream, _ptr(w), n_out, k_in, n_keep, m_group, _ptr(o.get("mask")),
+               _ptr(o["codes"]), _ptr(o.get("w_i8")), _ptr(o.get("sp_values")), _ptr(o.get("sp_meta")),
+               _ptr(o["w_scale"]), _ptr(workspace), workspace.numel())
     check(st, "bitlinear_quant_mask")
     o["workspace"] = workspace
     return o
@@ -145,10 +152,9 @@ def bitlinear_sgd_quant_mask(w: torch.Tensor, grad_w: torch.Tensor, lr: float, n
     if workspace is None:
         workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
     _need_bytes(workspace, ws_bytes, "workspace", dev)
-    st = lib().bitlinear_sgd_quant_mask(_ptr(w), _ptr(grad_w), float(lr), n_out, k_in, n_keep, m_group,
-                                        _ptr(o.get("mask")), _ptr(o["codes"]), _ptr(o.get("w_i8")),
-                                        _ptr(o.get("sp_values")), _ptr(o.get("sp_meta")), _ptr(o["w_scale"]),
-                                        _ptr(workspace), workspace.numel(), _stream(stream))
+    st = _call(lib().bitlinear_sgd_quant_mask, dev, stream, _ptr(w), _ptr(grad_w), float(lr), n_out, k_in, n_keep,
+               m_group, _ptr(o.get("mask")), _ptr(o["codes"]), _ptr(o.get("w_i8")), _ptr(o.get("sp_values")),
+               _ptr(o.get("sp_meta")), _ptr(o["w_scale"]), _ptr(workspace), workspace.numel())
     check(st, "bitlinear_sgd_quant_mask")
     o["workspace"] = workspace
     return o
@@ -156,7 +162,8 @@ def bitlinear_sgd_quant_mask(w: torch.Tensor, grad_w: torch.Tensor, lr: float, n
 
 def bitlinear_quant_mask_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise and return the range status (0 or BL_ERR_RANGE = -4); no raise."""
-    return int(lib().bitlinear_quant_mask_status(_ptr(workspace), _stream(stream)))
+    _need(workspace, torch.uint8, None, "workspace")
+    return _call(lib().bitlinear_quant_mask_status, workspace.device, stream, _ptr(workspace))
 
 
 def bitlinear_quant_mask_noalloc(w: torch.Tensor, n_keep: int, m_group: int, *, out: dict, stream=None) -> dict:
@@ -172,9 +179,8 @@ def bitlinear_quant_mask_noalloc(w: torch.Tensor, n_keep: int, m_group: int, *, 
     if m_group not in (4, 8) or k_in % m_group:
         raise ValueError(f"m_group must be 4 or 8 and divide k_in (got {m_group})")
     _check_qm_outputs(out, n_out, k_in, m_group, w.device)
-    st = lib().bitlinear_quant_mask_noalloc(_ptr(w), n_out, k_in, n_keep, m_group, _ptr(out.get("mask")),
-                                            _ptr(out["codes"]), _ptr(out.get("w_i8")), _ptr(out["w_scale"]),
-                                            _stream(stream))
+    st = _call(lib().bitlinear_quant_mask_noalloc, w.device, stream, _ptr(w), n_out, k_in, n_keep, m_group,
+               _ptr(out.get("mask")), _ptr(out["codes"]), _ptr(out.get("w_i8")), _ptr(out["w_scale"]))
     check(st, "bitlinear_quant_mask_noalloc")
     return out
 
@@ -190,7 +196,7 @@ def bitlinear_act_quant(x: torch.Tensor, *, xq: torch.Tensor | None = None, absm
         absmax = torch.empty((max(t, 1) + 3) // 4 * 4, dtype=torch.float32, device=x.device)[:t]
     _need(xq, torch.int8, (t, k_in), "xq", x.device)
     _need_vec(absmax, torch.float32, t, "absmax", x.device)
-    st = lib().bitlinear_act_quant(_ptr(x), t, k_in, _ptr(xq), _ptr(absmax), _stream(stream))
+    st = _call(lib().bitlinear_act_quant, x.device, stream, _ptr(x), t, k_in, _ptr(xq), _ptr(absmax))
     check(st, "bitlinear_act_quant")
     return xq, absmax
 
@@ -233,8 +239,8 @@ def bitlinear_fwd(xq: torch.Tensor, absmax: torch.Tensor, w_scale: torch.Tensor,
     if acc is not None:
         _need(acc, torch.int32, (t, n_out), "acc", dev)
     ydt = BL_OUT_F32 if y.dtype == torch.float32 else BL_OUT_BF16
-    st = lib().bitlinear_fwd(_ptr(xq), _ptr(absmax), _ptr(codes), _ptr(w_i8), _ptr(sp_values), _ptr(sp_meta),
-                             _ptr(w_scale), t, k_in, n_out, _ptr(acc), _ptr(y), ydt, _stream(stream))
+    st = _call(lib().bitlinear_fwd, dev, stream, _ptr(xq), _ptr(absmax), _ptr(codes), _ptr(w_i8), _ptr(sp_values),
+               _ptr(sp_meta), _ptr(w_scale), t, k_in, n_out, _ptr(acc), _ptr(y), ydt)
     check(st, "bitlinear_fwd")
     return y, acc
 
@@ -246,13 +252,15 @@ def bitlinear_fwd_grouped(problems: list[dict], *, y_dtype=torch.bfloat16, strea
     optionally ``y``, ``acc`` (outputs allocated here when missing, ``want_acc`` to
     request the int32 accumulators). Returns the dicts with ``y`` (and ``acc``) set.
     """
-    arr = (_lib.BlFwdProblem * max(1, len(problems)))()
+    if not problems:
+        return []
+    arr = (_lib.BlFwdProblem * len(problems))()
     out = []
+    dev = problems[0]["xq"].device
     for i, p in enumerate(problems):
         xq, codes = p["xq"], p["codes"]
-        _need(xq, torch.int8, None, f"problem {i} xq")
+        _need(xq, torch.int8, None, f"problem {i} xq", dev)
         t, k_in = xq.shape
-        dev = xq.device
         n_out = codes.shape[0]
         _need(codes, torch.uint8, (n_out, k_in // 4), f"problem {i} codes", dev)
         _need_vec(p["absmax"], torch.float32, t, f"problem {i} absmax", dev)
@@ -270,7 +278,7 @@ def bitlinear_fwd_grouped(problems: list[dict], *, y_dtype=torch.bfloat16, strea
                                    _ptr(acc), _ptr(y))
         out.append({**p, "y": y, "acc": acc})
     ydt = BL_OUT_F32 if y_dtype == torch.float32 else BL_OUT_BF16
-    st = lib().bitlinear_fwd_grouped(arr, len(problems), ydt, _stream(stream))
+    st = _call(lib().bitlinear_fwd_grouped, dev, stream, arr, len(problems), ydt)
     check(st, "bitlinear_fwd_grouped")
     return out
 
@@ -302,7 +310,7 @@ def bitlinear_grad_w_grouped(problems: list[dict], *, grad_w_dtype=torch.bfloat1
         arr[i] = _lib.BlGradWProblem(_ptr(dy), _ptr(x), k_in, n_out, _ptr(gw),
                                      BL_OUT_F32 if grad_w_dtype == torch.float32 else BL_OUT_BF16)
         out.append(gw)
-    st = lib().bitlinear_grad_w_grouped(arr, len(problems), t, _stream(stream))
+    st = _call(lib().bitlinear_grad_w_grouped, dev, stream, arr, len(problems), t)
     check(st, "bitlinear_grad_w_grouped")
     return out
 
@@ -361,9 +369,9 @@ def bitlinear_bwd(dy: torch.Tensor, x: torch.Tensor | None, codes: torch.Tensor 
         workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
     if workspace is not None:
         _need_bytes(workspace, need, "workspace", dev)
-    st = lib().bitlinear_bwd(_ptr(dy), _ptr(x), _ptr(xq), _ptr(absmax), _ptr(codes), _ptr(w_scale), t, k_in, n_out,
-                             _ptr(grad_x), _ptr(grad_w), gwdt, int(flags), _ptr(workspace),
-                             0 if workspace is None else workspace.numel(), _stream(stream))
+    st = _call(lib().bitlinear_bwd, dev, stream, _ptr(dy), _ptr(x), _ptr(xq), _ptr(absmax), _ptr(codes),
+               _ptr(w_scale), t, k_in, n_out, _ptr(grad_x), _ptr(grad_w), gwdt, int(flags), _ptr(workspace),
+               0 if workspace is None else workspace.numel())
     check(st, "bitlinear_bwd")
     return grad_x, grad_w
 
@@ -379,13 +387,13 @@ def bitlinear_grad_x_i8(dy: torch.Tensor, codes: torch.Tensor, w_scale: torch.Te
     {"grad_x", "acc" (or None)}."""
     t, n_out = dy.shape
     _need(dy, torch.bfloat16, None, "dy")
+    dev = dy.device
     if k_in is None:
         k_in = codes.shape[1] * 4
-    _need(codes, torch.uint8, (n_out, k_in // 4), "codes")
-    dev = dy.device
+    _need(codes, torch.uint8, (n_out, k_in // 4), "codes", dev)
     if grad_x is None:
         grad_x = torch.empty((t, k_in), dtype=torch.bfloat16, device=dev)
-    _need(grad_x, torch.bfloat16, (t, k_in), "grad_x")
+    _need(grad_x, torch.bfloat16, (t, k_in), "grad_x", dev)
     acc = torch.empty((t, k_in), dtype=torch.int32, device=dev) if want_acc else None
     _need_vec(w_scale, torch.float32, 1, "w_scale", dev)
     need = bitlinear_grad_x_i8_workspace_size(t, k_in, n_out)
@@ -393,8 +401,8 @@ def bitlinear_grad_x_i8(dy: torch.Tensor, codes: torch.Tensor, w_scale: torch.Te
         workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
     if workspace is not None:
         _need_bytes(workspace, need, "workspace", dev)
-    st = lib().bitlinear_grad_x_i8(_ptr(dy), _ptr(codes), _ptr(w_scale), t, k_in, n_out, _ptr(grad_x), _ptr(acc),
-                                   _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream))
+    st = _call(lib().bitlinear_grad_x_i8, dev, stream, _ptr(dy), _ptr(codes), _ptr(w_scale), t, k_in, n_out,
+               _ptr(grad_x), _ptr(acc), _ptr(workspace), 0 if workspace is None else workspace.numel())
     check(st, "bitlinear_grad_x_i8")
     return {"grad_x": grad_x, "acc": acc}
 
@@ -412,14 +420,14 @@ def bitlinear_mask_threshold_hist(w: torch.Tensor, mask: torch.Tensor, w_scale: 
     if out is None:
         out = torch.empty((19,), dtype=torch.int64, device=w.device)
     _need(out, torch.int64, (19,), "out", w.device)
-    st = lib().bitlinear_mask_threshold_hist(_ptr(w), _ptr(mask), _ptr(w_scale), n_out, k_in, m_group, _ptr(out),
-                                             _stream(stream))
+    st = _call(lib().bitlinear_mask_threshold_hist, w.device, stream, _ptr(w), _ptr(mask), _ptr(w_scale), n_out,
+               k_in, m_group, _ptr(out))
     check(st, "bitlinear_mask_threshold_hist")
     return out
 
 
 def bitlinear_device_status() -> tuple[int, int]:
-    """(status, bits): synchronise the device and read/clear the library's timeout bits."""
+    """(status, bits): synchronise the current device and read/clear the library's timeout bits."""
     bits = ctypes.c_uint(0)
     st = lib().bitlinear_device_status(ctypes.byref(bits))
     return int(st), int(bits.value)

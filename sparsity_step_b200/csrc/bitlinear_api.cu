@@ -24,10 +24,12 @@ namespace {
 thread_local char g_err[512] = "";
 
 bl_status fail(bl_status st, const char* fmt, ...) {
+  char msg[sizeof(g_err)];   // formatted apart from g_err: an argument may be g_err itself
   va_list ap;
   va_start(ap, fmt);
-  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  vsnprintf(msg, sizeof(msg), fmt, ap);
   va_end(ap);
+  memcpy(g_err, msg, sizeof(g_err));
   return st;
 }
 

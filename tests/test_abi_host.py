@@ -136,7 +136,7 @@ def test_fwd_grouped_validation(L):
     assert L.bitlinear_fwd_grouped(arr, 2, 5, None) == -1
     arr[1].k_in = 100
     assert L.bitlinear_fwd_grouped(arr, 2, 0, None) == -2
-    assert "problem 1" in _err(L)
+    assert _err(L).startswith("problem 1: k_in=100")   # the shape message kept inside the problem's
     arr[1].k_in = 2048
     arr[1].codes = None
     assert L.bitlinear_fwd_grouped(arr, 2, 0, None) == -1
@@ -225,3 +225,41 @@ def test_ctypes_signatures_match_header_arity():
         params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
         assert len(params) == len(args), name
     assert ctypes.sizeof(ctypes.c_size_t) == 8
+
+
+def test_binding_calls_on_the_tensors_device(monkeypatch):
+    """Every library call runs with the tensors' device current and that device's stream
+    as its last argument; a stream of another device is refused before the call."""
+    import contextlib
+
+    import torch
+
+    from sparsity_step_b200 import bitlinear as B
+
+    made_current, asked = [], []
+
+    @contextlib.contextmanager
+    def fake_device(dev):
+        made_current.append(dev)
+        yield
+
+    class FakeStream:
+        def __init__(self, dev, handle):
+            self.device, self.cuda_stream = dev, handle
+
+    def fake_current_stream(dev=None):
+        asked.append(dev)
+        return FakeStream(dev, 0x5000 + dev.index)
+
+    monkeypatch.setattr(torch.cuda, "device", fake_device)
+    monkeypatch.setattr(torch.cuda, "current_stream", fake_current_stream)
+    seen = []
+    fn = lambda *a: seen.append(a) or 0   # noqa: E731
+    d1 = torch.device("cuda", 1)
+    assert B._call(fn, d1, None, 7, 8) == 0
+    assert made_current == [d1] and asked == [d1] and seen == [(7, 8, 0x5001)]
+    assert B._call(fn, d1, FakeStream(d1, 0x77), 9) == 0
+    assert seen[-1] == (9, 0x77)
+    with pytest.raises(ValueError, match="stream is on"):
+        B._call(fn, d1, FakeStream(torch.device("cuda", 0), 0x66), 9)
+    assert len(seen) == 2 and made_current == [d1, d1]
