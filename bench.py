@@ -166,6 +166,20 @@ class RankSync:
         return float(t.item())
 
 
+def choose_bf16_peak(peaks: dict, clocks: dict, ms_total: float) -> tuple[float, bool, str]:
+    """The bf16 roofline denominator for kernels timed inside the step: the measured
+    burst rate when the median SM clock under load stayed within 5 % of its maximum
+    (the clock the burst figure was taken at), else the sustained (power-capped) rate.
+    Without a clock record, a timed region under a second counts as a burst.
+    Returns (peak TFLOP/s, burst?, the reason in words)."""
+    smhz, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    at_max_clock = bool(smhz and smax and smhz >= 0.95 * smax)
+    use_burst = at_max_clock if (smhz and smax) else ms_total < 1000.0
+    peak = peaks["bf16_tflops"] if use_burst else peaks["bf16_tflops_sustained"]
+    why = "timed region %.0f ms, median SM clock %s of max %s MHz" % (ms_total, smhz, smax)
+    return peak, use_burst, why
+
+
 def job_tokens_per_s(ms_per_step: float, world: int) -> float:
     """Whole-job throughput: every rank processes its own TOKENS per step (weak
     scaling); the step time is the max over ranks."""
@@ -447,22 +461,14 @@ def run_ours(args) -> None:
     except (OSError, RuntimeError) as exc:
         probe = {"error": str(exc)}
 
-    # ---------------- roofline of the dominant kernel
-    # Peak: the measured burst bf16 rate when the SM clock stayed near its maximum (the
-    # kernels ran at the clock the burst figure was taken at); the sustained
-    # (power-capped) rate when the power cap lowered the clock during the timed region.
-    # Without a clock record, a region under a second counts as a burst.
+    # ---------------- roofline of the dominant kernel (burst or sustained peak by clock)
     peaks = load_peaks()
+    bf16_peak, use_burst, why = choose_bf16_peak(peaks, clocks, ms_total)
     fwd_ops, bwd_flops = algorithmic_counts()
     gemm_flops = 2 * TOKENS * 2048 * 11008          # every product here has this size
     # one bwd_grad_w launch computes all three weight gradients; a bwd_grad_x call is one
     # product (its time includes the 2-bit code expansion that feeds it)
     flops_per_launch = {"bwd_grad_w": 3 * gemm_flops, "bwd_grad_x": gemm_flops}
-    smhz, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
-    at_max_clock = bool(smhz and smax and smhz >= 0.95 * smax)
-    use_burst = at_max_clock if (smhz and smax) else ms_total < 1000.0
-    bf16_peak = peaks["bf16_tflops"] if use_burst else peaks["bf16_tflops_sustained"]
-    why = ("timed region %.0f ms, median SM clock %s of max %s MHz" % (ms_total, smhz, smax))
 
     def gemm_roofline(cls):
         achieved = flops_per_launch[cls] / (per_launch_ms[cls] * 1e-3) / 1e12
