@@ -147,17 +147,16 @@ bl_status bitlinear_quant_mask_status(const void* workspace, void* stream);
  * (which may synchronise the device) are not allowed.
  *
  * Same computation, arguments and outputs as bitlinear_quant_mask, minus the
- * workspace and the 2:4 outputs. Its scratch is a fixed array of 19200 bytes inside the library (every
- * GPU that loads the library holds it until exit), which limits the tensor to
- * n_out * k_in <= 4966055936 weights; larger tensors get BL_ERR_UNSUPPORTED_SHAPE.
- * The first call on each device looks up that array's device address (with the
- * device current) and keeps it for the life of the process; make that first call
- * before any stream capture. A reset of the device's primary context
- * (cudaDeviceReset) invalidates the kept address: do not call this entry point on a
- * device after resetting it. All calls on a
- * device share the array, so calls that overlap on the GPU race: order them on one
- * stream. A range error shows as gamma = NaN and all-zero codes (there is no
- * workspace to read a status from).
+ * workspace and the 2:4 outputs. Its scratch is a fixed array of 19200 bytes inside
+ * the library (every GPU that loads the library holds it until exit), which limits
+ * the tensor to n_out * k_in <= 4966055936 weights; larger tensors get
+ * BL_ERR_UNSUPPORTED_SHAPE. The first call on each device looks up that array's
+ * device address (with the device current) and keeps it for the life of the process;
+ * make that first call before any stream capture. A reset of the device's primary
+ * context (cudaDeviceReset) invalidates the kept address: do not call this entry
+ * point on a device after resetting it. All calls on a device share the array, so
+ * calls that overlap on the GPU race: order them on one stream. A range error shows
+ * as gamma = NaN and all-zero codes (there is no workspace to read a status from).
  */
 bl_status bitlinear_quant_mask_noalloc(const float* w_latent, int64_t n_out, int64_t k_in, int n_keep, int m_group,
                                        uint8_t* mask_out, uint8_t* codes_out, int8_t* w_i8_out, float* w_scale_out,
@@ -221,8 +220,8 @@ typedef struct {
  * a layer stack at one decode step, or the q/k/v or gate/up linears that share an
  * input). Same result as bitlinear_fwd with the codes operand for each problem; the
  * packed 2-bit codes are streamed once per 128 tokens (once per 8 tokens when the
- * largest problem has at most 8). `problems` is a HOST array
- * (copied into the launch); y_dtype applies to all problems. Problems may have t = 0.
+ * largest problem has at most 8). `problems` is a HOST array (copied into the
+ * launch); y_dtype applies to all problems. Problems may have t = 0.
  * The one-time layout check of bitlinear_fwd applies here too (batches of up to 8).
  * More than 256 problems: BL_ERR_UNSUPPORTED_SHAPE.
  */
