@@ -263,3 +263,30 @@ def test_binding_calls_on_the_tensors_device(monkeypatch):
     with pytest.raises(ValueError, match="stream is on"):
         B._call(fn, d1, FakeStream(torch.device("cuda", 0), 0x66), 9)
     assert len(seen) == 2 and made_current == [d1, d1]
+
+
+def test_binding_checks_buffers_before_the_library():
+    """Host tensors, wrong dtypes and missing operands are refused in Python, before any
+    pointer reaches the library (no CUDA call is made)."""
+    import torch
+
+    from sparsity_step_b200 import bitlinear as B
+
+    w = torch.zeros((16, 64), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        B.bitlinear_quant_mask(w, 6, 8)
+    with pytest.raises(TypeError, match="float32"):
+        B.bitlinear_quant_mask(w.double(), 6, 8)
+    with pytest.raises(TypeError, match="bfloat16"):
+        B.bitlinear_act_quant(torch.zeros((4, 64), dtype=torch.float16))
+    xq = torch.zeros((4, 64), dtype=torch.int8)
+    a = torch.ones(4)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        B.bitlinear_fwd(xq, a, torch.ones(1), w_i8=torch.zeros((16, 64), dtype=torch.int8))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        B.bitlinear_fwd(xq, a, torch.ones(1))   # the dtype/device check of xq comes first
+    with pytest.raises(ValueError, match="1 to 4"):
+        B.bitlinear_grad_w_grouped([])
+    assert B.bitlinear_fwd_grouped([]) == []
+    with pytest.raises(TypeError, match="torch.Tensor"):
+        B._need([1, 2], torch.int8, None, "x")
