@@ -22,6 +22,9 @@ def _call(fn, dev: torch.device, stream, *args) -> int:
     the stream (last argument) is the given one or that device's current stream."""
     if stream is not None and stream.device != dev:
         raise ValueError(f"stream is on {stream.device}, the tensors on {dev}")
+    if torch.cuda.current_device() == dev.index:   # the usual case: no device switch
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        return int(fn(*args, int(s.cuda_stream)))
     with torch.cuda.device(dev):
         s = torch.cuda.current_stream(dev) if stream is None else stream
         return int(fn(*args, int(s.cuda_stream)))

@@ -251,18 +251,24 @@ def test_binding_calls_on_the_tensors_device(monkeypatch):
         asked.append(dev)
         return FakeStream(dev, 0x5000 + dev.index)
 
+    current = [0]
     monkeypatch.setattr(torch.cuda, "device", fake_device)
     monkeypatch.setattr(torch.cuda, "current_stream", fake_current_stream)
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: current[0])
     seen = []
     fn = lambda *a: seen.append(a) or 0   # noqa: E731
-    d1 = torch.device("cuda", 1)
+    d0, d1 = torch.device("cuda", 0), torch.device("cuda", 1)
+    # tensors on another device than the current one: switched for the call
     assert B._call(fn, d1, None, 7, 8) == 0
     assert made_current == [d1] and asked == [d1] and seen == [(7, 8, 0x5001)]
     assert B._call(fn, d1, FakeStream(d1, 0x77), 9) == 0
     assert seen[-1] == (9, 0x77)
     with pytest.raises(ValueError, match="stream is on"):
-        B._call(fn, d1, FakeStream(torch.device("cuda", 0), 0x66), 9)
+        B._call(fn, d1, FakeStream(d0, 0x66), 9)
     assert len(seen) == 2 and made_current == [d1, d1]
+    # tensors on the current device: no switch, that device's stream
+    assert B._call(fn, d0, None, 5) == 0
+    assert seen[-1] == (5, 0x5000) and made_current == [d1, d1] and asked[-1] == d0
 
 
 def test_binding_checks_buffers_before_the_library():
