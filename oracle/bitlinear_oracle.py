@@ -1,7 +1,8 @@
 """CPU oracle of the Sparse-BitNet BitLinear path: plain, slow, obviously correct.
 
 TEST INFRASTRUCTURE. Only the tests, the smoke check of ``__graft_entry__`` and the
-CPU-baseline leg of ``bench.py`` may import this module. The product path (the
+CPU legs of ``bench.py`` (``cpu_baseline`` and ``--impl reference``) may import this
+module. The product path (the
 CUDA library and its Python binding) never imports, calls or falls back to it,
 and this module imports nothing from the product package.
 
