@@ -228,7 +228,7 @@ void set_raster(bl::GemmArgs& g, double a_bytes, double b_bytes) {
 // (bl::kDecLutAddr) below which its first ring slot must fit. Where the dynamic shared
 // memory starts depends on the device and the driver, so the first launch on each device
 // runs one CTA of the kernel in probe mode, reads that address back (synchronously: the
-// first call must not be under stream capture) and remembers the verdict. A device
+// first call must not be under stream capture) and remembers the result. A device
 // where the table does not fit gets BL_ERR_CUDA from every call, before anything is
 // enqueued, instead of a launch that would leave y unwritten.
 constexpr int kMaxLayoutDevices = 64;
