@@ -63,3 +63,25 @@ def test_reference_arm_only_rank0_prints(monkeypatch):
     with redirect_stdout(buf):
         bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
     assert buf.getvalue() == ""
+
+
+def test_reference_arm_line_on_rank0(monkeypatch):
+    """The oracle arm's JSON line carries the contract's keys, its own cpu_baseline and a
+    zero-copy e2e, with value = the sample's tokens / the measured step time."""
+    import json
+
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert abs(line["value"] - bench.SAMPLE_TOKENS / (line["ms_per_step"] * 1e-3)) <= 0.01 * line["value"]
